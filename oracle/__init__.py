@@ -1,0 +1,33 @@
+"""CPU oracle for the block-draft hot path -- TEST INFRASTRUCTURE ONLY.
+
+A plain, slow, obviously correct float64 restatement of what the path
+computes, written from the DFlash 2 pages ("DFlash 2: Keep Drafting Parallel",
+the Chinese translation of the blog, and "Inco AI's DFlash 2 lifts LLM decoding
+output 16-25%") plus the stand-in scorer and walk that this library fixes where
+the pages leave the computation open.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import or run anything here.  The CUDA library never calls
+it, shares no code with it, and has no CPU fallback.
+
+Inputs are the same bf16 bit patterns (np.uint16) the GPU path receives; the
+oracle widens them exactly to float64 and computes the plain definitions with
+no blocking, fusion or reordering beyond what each definition states.
+
+Pins (``tests/test_oracle_*.py``, run with ``-m "not gpu"``):
+  conv2tap      hand-worked case, identity/shift taps, marker inputs
+  lmhead_topk   exact rational/decimal brute force on tiny shapes, heap
+                selection, the uniform-logit case (lse = log V)
+  argmax_tokens exact brute force, tie to the lowest index
+  pair_scores / viterbi / path_select
+                exhaustive 16^L enumeration for L <= 4 on an exact rational
+                pair table, the E = 0 case (= the top-1 path), a hand case
+  verify        hand cases and the Table 1 closed form (4.27 / 6.79)
+"""
+from .conv import conv2tap
+from .lmhead import logits, lmhead_topk, argmax_tokens, topk_margin_ok
+from .selector import pair_scores, viterbi, viterbi_two_best, path_select
+from .verify import verify
+
+__all__ = ["conv2tap", "logits", "lmhead_topk", "argmax_tokens", "topk_margin_ok",
+           "pair_scores", "viterbi", "viterbi_two_best", "path_select", "verify"]

@@ -1,0 +1,30 @@
+"""Block-draft hot path on B200 (sm_100a): two-tap conv, fused LM-head top-16,
+pair-score path selection, greedy verification.
+
+The compute lives in libdflash.so (C ABI in include/dflash.h); this package is
+the thin ctypes binding over it.  Importing it fails loudly when the library
+has not been built: there is no CPU fallback.
+"""
+import numpy as np
+import torch
+
+from ._binding import (  # noqa: F401
+    DFlashError,
+    K_TOP,
+    LIB_PATH,
+    dflash_conv2tap,
+    dflash_lmhead_logits_debug,
+    dflash_lmhead_topk,
+    dflash_lmhead_topk_workspace,
+    dflash_path_select,
+    dflash_status_string,
+    dflash_verify,
+    lib,
+    workspace,
+)
+
+
+def bf16_tensor(bits: np.ndarray, device="cuda") -> torch.Tensor:
+    """Wrap bf16 bit patterns (np.uint16) as a torch.bfloat16 tensor on `device`."""
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+    return t.to(device) if device is not None else t

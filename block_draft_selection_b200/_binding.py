@@ -1,0 +1,192 @@
+"""ctypes binding of libdflash.so: argument marshalling only.
+
+Each function here has the name of the C entry point it calls, checks that
+the torch tensors it is given are CUDA tensors of the layout the C ABI
+documents (include/dflash.h), allocates outputs the caller did not pass, and
+forwards raw device pointers and the current CUDA stream.  Every step of the
+computation runs in the library's kernels; there is no CPU path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdflash.so")
+
+DFLASH_OK = 0
+DFLASH_ERR_INVALID_ARG = 1
+DFLASH_ERR_UNSUPPORTED = 2
+DFLASH_ERR_CUDA = 3
+DFLASH_ERR_WORKSPACE = 4
+DFLASH_ERR_TIMEOUT = 5
+DFLASH_ERR_BAD_INDEX = 6
+K_TOP = 16
+
+
+class DFlashError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn}: {dflash_status_string(code)} (status {code})")
+        self.code = code
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m block_draft_selection_b200.build` "
+            "(this package has no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    sig = {
+        "dflash_status_string": (ctypes.c_char_p, [i32]),
+        "dflash_conv2tap": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, vp]),
+        "dflash_lmhead_topk_workspace": (sz, [i32, i32, i32]),
+        "dflash_lmhead_topk": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, sz, vp, vp]),
+        "dflash_lmhead_logits_debug": (i32, [vp, vp, i32, i32, i32, vp, vp, sz, vp, vp]),
+        "dflash_path_select": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]),
+        "dflash_verify": (i32, [vp, vp, i32, i32, vp, vp, vp]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def dflash_status_string(code: int) -> str:
+    return lib.dflash_status_string(int(code)).decode()
+
+
+def _check(fn: str, code: int):
+    if code != DFLASH_OK:
+        raise DFlashError(fn, code)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, name, dtype, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def _out(t, name, dtype, shape, device):
+    if t is None:
+        return torch.empty(shape, dtype=dtype, device=device)
+    return _need(t, name, dtype, shape)
+
+
+def dflash_conv2tap(x, a0, a1, prev=None, y=None, stream=None):
+    """y[b,t,c] = a0[c] x[b,t,c] + a1[c] x[b,t-1,c], x[b,-1,:] = prev[b,:] (zeros if None).
+    x [B,P,d] bf16; a0, a1 [d] bf16; prev [B,d] bf16 or None."""
+    _need(x, "x", torch.bfloat16)
+    B, P, d = x.shape
+    _need(a0, "a0", torch.bfloat16, (d,))
+    _need(a1, "a1", torch.bfloat16, (d,))
+    if prev is not None:
+        _need(prev, "prev", torch.bfloat16, (B, d))
+    y = _out(y, "y", torch.bfloat16, (B, P, d), x.device)
+    _check("dflash_conv2tap", lib.dflash_conv2tap(_ptr(x), _ptr(prev), _ptr(a0), _ptr(a1), _ptr(y),
+                                                  B, P, d, _stream(stream)))
+    return y
+
+
+def dflash_lmhead_topk_workspace(M: int, V: int, d: int) -> int:
+    return int(lib.dflash_lmhead_topk_workspace(M, V, d))
+
+
+def workspace(M: int, V: int, d: int, device="cuda") -> torch.Tensor:
+    n = dflash_lmhead_topk_workspace(M, V, d)
+    if n == 0:
+        raise DFlashError("dflash_lmhead_topk_workspace", DFLASH_ERR_INVALID_ARG)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def dflash_lmhead_topk(H, W, K=K_TOP, topk_logp=None, topk_idx=None, lse=None, ws=None,
+                       dev_status=None, stream=None, want_lse=True):
+    """H [M,d] bf16, W [V,d] bf16 -> (topk_logp [M,16] f32, topk_idx [M,16] i32, lse [M] f32)."""
+    _need(H, "H", torch.bfloat16)
+    _need(W, "W", torch.bfloat16)
+    M, d = H.shape
+    V = W.shape[0]
+    if W.shape[1] != d:
+        raise ValueError("H and W disagree on d")
+    topk_logp = _out(topk_logp, "topk_logp", torch.float32, (M, K), H.device)
+    topk_idx = _out(topk_idx, "topk_idx", torch.int32, (M, K), H.device)
+    if lse is None and want_lse:
+        lse = torch.empty(M, dtype=torch.float32, device=H.device)
+    elif lse is not None:
+        _need(lse, "lse", torch.float32, (M,))
+    if ws is None:
+        ws = workspace(M, V, d, H.device)
+    if dev_status is not None:
+        _need(dev_status, "dev_status", torch.int32, (1,))
+    _check("dflash_lmhead_topk", lib.dflash_lmhead_topk(
+        _ptr(H), _ptr(W), M, V, d, K, _ptr(topk_logp), _ptr(topk_idx), _ptr(lse), _ptr(ws),
+        ws.numel(), _ptr(dev_status), _stream(stream)))
+    return topk_logp, topk_idx, lse
+
+
+def dflash_lmhead_logits_debug(H, W, z=None, ws=None, dev_status=None, stream=None):
+    """Raw logits z [M,V] f32 through the same GEMM path (diagnostic)."""
+    _need(H, "H", torch.bfloat16)
+    _need(W, "W", torch.bfloat16)
+    M, d = H.shape
+    V = W.shape[0]
+    z = _out(z, "z", torch.float32, (M, V), H.device)
+    if ws is None:
+        ws = workspace(M, V, d, H.device)
+    _check("dflash_lmhead_logits_debug", lib.dflash_lmhead_logits_debug(
+        _ptr(H), _ptr(W), M, V, d, _ptr(z), _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream)))
+    return z
+
+
+def dflash_path_select(topk_logp, topk_idx, E, Msel, B, L, path_tok=None, path_slot=None,
+                       path_score=None, pair_scores=False, dev_status=None, stream=None):
+    """Returns (path_tok [B,L] i32, path_slot [B,L] i32, path_score [B] f32, pair scores
+    [B,L-1,16,16] f32 or None)."""
+    _need(topk_logp, "topk_logp", torch.float32, (B * L, K_TOP))
+    _need(topk_idx, "topk_idx", torch.int32, (B * L, K_TOP))
+    _need(E, "E", torch.bfloat16)
+    V, r = E.shape
+    _need(Msel, "Msel", torch.bfloat16, (r, r))
+    dev = topk_logp.device
+    path_tok = _out(path_tok, "path_tok", torch.int32, (B, L), dev)
+    path_slot = _out(path_slot, "path_slot", torch.int32, (B, L), dev)
+    path_score = _out(path_score, "path_score", torch.float32, (B,), dev)
+    pair = torch.empty((B, max(L - 1, 0), K_TOP, K_TOP), dtype=torch.float32, device=dev) if pair_scores else None
+    _check("dflash_path_select", lib.dflash_path_select(
+        _ptr(topk_logp), _ptr(topk_idx), _ptr(E), _ptr(Msel), B, L, K_TOP, r, V, _ptr(path_tok),
+        _ptr(path_slot), _ptr(path_score), _ptr(pair) if pair is not None and pair.numel() else None,
+        _ptr(dev_status), _stream(stream)))
+    return path_tok, path_slot, path_score, pair
+
+
+def dflash_verify(draft, target, accept_len=None, next_token=None, stream=None):
+    """draft [B,L] i32, target [B,L+1] i32 -> (accept_len [B] i32, next_token [B] i32)."""
+    _need(draft, "draft", torch.int32)
+    B, L = draft.shape
+    _need(target, "target", torch.int32, (B, L + 1))
+    accept_len = _out(accept_len, "accept_len", torch.int32, (B,), draft.device)
+    next_token = _out(next_token, "next_token", torch.int32, (B,), draft.device)
+    _check("dflash_verify", lib.dflash_verify(_ptr(draft), _ptr(target), B, L, _ptr(accept_len),
+                                              _ptr(next_token), _stream(stream)))
+    return accept_len, next_token

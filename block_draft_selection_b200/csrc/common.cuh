@@ -1,0 +1,301 @@
+// Shared device helpers for the sm_100a kernels: status words, bounded
+// mbarrier waits, TMA tile loads, tcgen05 (TMEM / UMMA) wrappers.
+//
+// Every wait here is bounded by a deadline on %globaltimer.  A wait that runs
+// out records DFLASH_ERR_TIMEOUT in the caller's status word and returns
+// false; the calling role then drains what it has in flight and leaves, so
+// no kernel in this library can spin forever.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/dflash.h"
+
+#ifndef __CUDACC_RTC__
+#include <cuda.h>
+#endif
+
+namespace dflash {
+
+// ---------------------------------------------------------------- status ---
+
+__device__ __forceinline__ void set_status(int* status, int code) {
+  if (status != nullptr) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// ---------------------------------------------------------------- mbarrier --
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile(
+      "{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(bar),
+      "r"(bytes)
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete, at most until
+// `deadline` (globaltimer ns) or until *abort becomes nonzero.  Returns false
+// (and records a timeout) when it gives up.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t deadline,
+                                          volatile int* abort, int* status) {
+  uint32_t spins = 0;
+  while (!mbar_try_wait(bar, parity)) {
+    if ((++spins & 63u) == 0) {
+      if (*abort) return false;
+      if (globaltimer_ns() > deadline) {
+        set_status(status, DFLASH_ERR_TIMEOUT);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+  return true;
+}
+
+// ---------------------------------------------------------------- TMA -------
+
+// 2-D tiled bulk tensor load global -> shared, completion counted in bytes on
+// `bar`.  c0 is the innermost (contiguous) coordinate in elements, c1 the row.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+// Same, with an L2 eviction-priority hint (a createpolicy value).
+__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                 int c0, int c1, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ---------------------------------------------------------------- tcgen05 ---
+
+// Shared-memory matrix descriptor for a K-major bf16 operand laid out by a
+// 128-byte-swizzled TMA load: rows of 128 bytes (64 bf16), 8-row swizzle
+// atoms of 1024 bytes stacked along M/N.  Fields (tcgen05 matrix descriptor):
+// [0,14) start address >> 4; [16,30) leading byte offset >> 4 (unused for
+// swizzled K-major, set to 1); [32,46) stride byte offset >> 4 (1024 B between
+// 8-row atoms); [46,48) descriptor version = 1; [49,52) base offset = 0
+// (atoms are 1024-byte aligned); [61,64) swizzle mode 2 = 128-byte.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1u) << 16;
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
+// Instruction descriptor for tcgen05.mma kind::f16 with bf16 A and B, fp32
+// accumulate, both operands K-major, dense: [4,6) D format (1 = f32);
+// [7,10) A format (1 = bf16); [10,13) B format (1 = bf16); bits 15/16 = 0
+// (K-major); [17,23) N >> 3; [24,29) M >> 4.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16_f32(int m, int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+         (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive once on `bar` when every tcgen05.mma issued so far by this thread
+// has completed (and its shared-memory operands may be overwritten).
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// TMEM allocation: executed by one full warp.  Writes the base address to
+// *dst_smem.  ncols is a power of two in [32, 512].
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// 32 lanes x 32 bits, 16 consecutive columns: thread t of the warp receives
+// TMEM lane (lane base + t), columns [col, col+16).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ int elect_lane0() { return (threadIdx.x & 31) == 0; }
+
+// ------------------------------------------------------ top-16 in registers --
+
+constexpr int KTOP = 16;
+
+// (value desc, index asc) strict order.
+__device__ __forceinline__ bool better(float a, int ia, float b, int ib) {
+  return a > b || (a == b && ia < ib);
+}
+
+// Running candidate list kept sorted in registers, plus an online
+// log-sum-exp state (m = running max, s = sum of exp(z - m)).
+struct TopState {
+  float v[KTOP];
+  int i[KTOP];
+  float m;
+  float s;
+
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int k = 0; k < KTOP; ++k) {
+      v[k] = -INFINITY;
+      i[k] = 0x7fffffff;
+    }
+    m = -INFINITY;
+    s = 0.f;
+  }
+
+  // Insert (x, ix) if it beats the current 16th entry under the full order.
+  __device__ __forceinline__ void insert(float x, int ix) {
+    if (!better(x, ix, v[KTOP - 1], i[KTOP - 1])) return;
+    v[KTOP - 1] = x;
+    i[KTOP - 1] = ix;
+#pragma unroll
+    for (int k = KTOP - 1; k > 0; --k) {
+      const bool sw = better(v[k], i[k], v[k - 1], i[k - 1]);
+      const float a = v[k], b = v[k - 1];
+      const int ia = i[k], ib = i[k - 1];
+      v[k - 1] = sw ? a : b;
+      v[k] = sw ? b : a;
+      i[k - 1] = sw ? ia : ib;
+      i[k] = sw ? ib : ia;
+    }
+  }
+
+  // Fold another (m, s) pair into this one.
+  __device__ __forceinline__ void merge_lse(float m2, float s2) {
+    if (m2 == -INFINITY) return;
+    if (m == -INFINITY) {
+      m = m2;
+      s = s2;
+      return;
+    }
+    const float mn = fmaxf(m, m2);
+    s = s * __expf(m - mn) + s2 * __expf(m2 - mn);
+    m = mn;
+  }
+
+  // Remove the head (entry 0), shifting the list up; the tail becomes empty.
+  __device__ __forceinline__ void pop_head() {
+#pragma unroll
+    for (int k = 0; k < KTOP - 1; ++k) {
+      v[k] = v[k + 1];
+      i[k] = i[k + 1];
+    }
+    v[KTOP - 1] = -INFINITY;
+    i[KTOP - 1] = 0x7fffffff;
+  }
+};
+
+// Partial record written per (row, slot) by the LM-head kernel and read by
+// the merge kernel: running max, sum of exp(z - max), 16 candidates.
+struct __align__(16) Partial {
+  float m;
+  float s;
+  float pad[2];
+  float v[KTOP];
+  int i[KTOP];
+};
+static_assert(sizeof(Partial) == 144, "partial record layout");
+
+}  // namespace dflash

@@ -1,0 +1,155 @@
+/*
+ * dflash.h -- C ABI of the block-draft hot path (sm_100a / B200).
+ *
+ * One draft cycle of a one-shot block drafter in four stages:
+ *   dflash_conv2tap     two-tap block-local convolution
+ *   dflash_lmhead_topk  LM head over the full vocabulary fused with
+ *                       log-softmax and per-position top-16 selection
+ *   dflash_path_select  pair scores of neighbouring candidates + max-sum walk
+ *   dflash_verify       greedy verification (accepted length, next token)
+ *
+ * Sources: "DFlash 2: Keep Drafting Parallel" (the blog, read in its Chinese
+ * translation) and "Inco AI's DFlash 2 lifts LLM decoding output 16-25%".
+ *
+ * Conventions shared by every entry point
+ *   - Pointers are device pointers owned by the caller unless a parameter
+ *     says "host".  The library allocates no memory and keeps no state
+ *     between calls, so calls on different streams are independent.
+ *   - bf16 values are passed as their 16-bit patterns (dflash_bf16).
+ *   - All arrays are row-major and contiguous.  Token rows of a batch of
+ *     B blocks with L drafted positions are ordered b*L + i.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy stream).
+ *     Calls only enqueue work; the return code covers host-side argument
+ *     checks and launch errors.  Errors found on the device (a bounded wait
+ *     that ran out, an out-of-range token index) are written with atomicCAS
+ *     into `dev_status` (a device int the caller zeroes; NULL = not recorded).
+ *   - Every device-side wait is bounded (default 2000 ms, environment
+ *     variable DFLASH_TIMEOUT_MS overrides); a kernel that gives up records
+ *     DFLASH_ERR_TIMEOUT and returns instead of hanging.
+ */
+#ifndef DFLASH_H_
+#define DFLASH_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t dflash_bf16;
+
+enum dflash_status {
+  DFLASH_OK = 0,
+  DFLASH_ERR_INVALID_ARG = 1,   /* null pointer, bad size, K != 16, ... */
+  DFLASH_ERR_UNSUPPORTED = 2,   /* valid request this build cannot run */
+  DFLASH_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed */
+  DFLASH_ERR_WORKSPACE = 4,     /* workspace smaller than required */
+  DFLASH_ERR_TIMEOUT = 5,       /* device: a bounded wait gave up */
+  DFLASH_ERR_BAD_INDEX = 6      /* device: a token index outside [0, V) */
+};
+
+/* Static text for a status code (never NULL). */
+const char* dflash_status_string(int status);
+
+/*
+ * Two-tap block-local convolution.
+ * "DFlash 2: Keep Drafting Parallel", section "a lightweight local
+ * convolution", formula Conv_k(x)_t = k_{t,0} * x_t + k_{t,1} * x_{t-1}, and
+ * Figure 4: each position mixes with its predecessor inside the block; the
+ * first position reads the last verified token's representation.  Here the
+ * taps are the static per-channel base taps a0, a1.
+ *
+ *   y[b,t,c] = a0[c] * x[b,t,c] + a1[c] * x[b,t-1,c],  x[b,-1,c] = prev[b,c]
+ *
+ * x    [B, P, d] bf16        prev [B, d] bf16 (NULL: zeros)
+ * a0   [d] bf16              a1   [d] bf16
+ * y    [B, P, d] bf16 out    (fp32 arithmetic, rounded to nearest even)
+ * Requires B, P, d >= 1 and d % 8 == 0 (16-byte rows); y must not overlap x.
+ */
+int dflash_conv2tap(const dflash_bf16* x, const dflash_bf16* prev, const dflash_bf16* a0,
+                    const dflash_bf16* a1, dflash_bf16* y, int B, int P, int d, void* stream);
+
+/*
+ * Bytes of device workspace dflash_lmhead_topk needs for these sizes
+ * (0 when the sizes are invalid).
+ */
+size_t dflash_lmhead_topk_workspace(int M, int V, int d);
+
+/*
+ * LM head + log-softmax + top-16 per row, without writing logits to memory.
+ * "DFlash 2: Keep Drafting Parallel", section "the right token is already in
+ * the candidates" and Table 1 (each drafted position keeps its 16 best
+ * candidates), section "a lightweight path selector" (the candidates are
+ * scored without another LM-head pass).
+ *
+ *   z[m,v] = sum_k H[m,k] * W[v,k]     (bf16 inputs, fp32 accumulation)
+ *   lse[m] = log sum_v exp(z[m,v])
+ *   topk_idx[m,:]  = the 16 largest z[m,:], value descending, ties to the
+ *                    lowest vocabulary index
+ *   topk_logp[m,k] = z[m, topk_idx[m,k]] - lse[m]
+ *
+ * H [M, d] bf16, W [V, d] bf16 (both K-major, 16-byte aligned base).
+ * topk_logp [M, 16] fp32 out, topk_idx [M, 16] int32 out, lse [M] fp32 out
+ * (NULL: not written).  ws: device workspace of at least
+ * dflash_lmhead_topk_workspace(M, V, d) bytes, 256-byte aligned; its contents
+ * need no initialisation.  K must be 16, d % 8 == 0, M >= 1, V >= 16.
+ * Two kernels run on `stream`: the fused GEMM + epilogue (tcgen05 / TMEM /
+ * TMA) and the cross-CTA merge of the per-CTA partial lists.
+ */
+int dflash_lmhead_topk(const dflash_bf16* H, const dflash_bf16* W, int M, int V, int d, int K,
+                       float* topk_logp, int32_t* topk_idx, float* lse, void* ws, size_t ws_bytes,
+                       int* dev_status, void* stream);
+
+/*
+ * Diagnostic: the same GEMM path as dflash_lmhead_topk, but writing the raw
+ * logits z [M, V] fp32 (row-major) instead of selecting.  Meant for small
+ * shapes in tests; not part of the fused hot path.
+ */
+int dflash_lmhead_logits_debug(const dflash_bf16* H, const dflash_bf16* W, int M, int V, int d,
+                               float* z, void* ws, size_t ws_bytes, int* dev_status, void* stream);
+
+/*
+ * Path selection over the candidate lists.
+ * "DFlash 2: Keep Drafting Parallel", section "a lightweight path selector":
+ * all adjacent candidate pairs are scored at once, then one serial walk over
+ * the precomputed scores picks the path.  The pages' trained scorer is not
+ * published; this entry point computes the stand-in
+ *
+ *   S_i[j,k] = lp[i,j] + lp[i+1,k] + e_{c_ij} . Msel . e_{c_{i+1,k}}
+ *
+ * and walks it with max-sum (Viterbi): delta_0 = 0,
+ * delta_{i+1}[k] = max_j delta_i[j] + S_i[j,k] (ties: lowest j); the path ends
+ * at argmax_k delta_{L-1}[k] (ties: lowest k).  L = 1: slot 0, score 0.
+ *
+ * topk_logp [B*L, 16] fp32, topk_idx [B*L, 16] int32 (values in [0, V))
+ * E [V, r] bf16, Msel [r, r] bf16;  r % 8 == 0, 8 <= r <= 128; 1 <= L <= 16.
+ * path_tok [B, L] int32 out; path_slot [B, L] int32 out (NULL: not written);
+ * path_score [B] fp32 out (NULL: not written); pair_scores_dbg
+ * [B, L-1, 16, 16] fp32 out (NULL: not written).  An index outside [0, V)
+ * records DFLASH_ERR_BAD_INDEX and is read as index 0.
+ */
+int dflash_path_select(const float* topk_logp, const int32_t* topk_idx, const dflash_bf16* E,
+                       const dflash_bf16* Msel, int B, int L, int K, int r, int V,
+                       int32_t* path_tok, int32_t* path_slot, float* path_score,
+                       float* pair_scores_dbg, int* dev_status, void* stream);
+
+/*
+ * Greedy verification.
+ * "DFlash 2: Keep Drafting Parallel", Table 1 caption: the accepted length
+ * includes the verifier's next token.  With n the first i where
+ * draft[b,i] != target[b,i] (n = L if none):
+ *   accept_len[b] = n + 1,  next_token[b] = target[b, n].
+ *
+ * draft [B, L] int32, target [B, L+1] int32 (the target's argmax tokens at
+ * the L drafted positions and the bonus position).  accept_len [B] int32 out,
+ * next_token [B] int32 out.  1 <= L <= 32.
+ */
+int dflash_verify(const int32_t* draft, const int32_t* target, int B, int L, int32_t* accept_len,
+                  int32_t* next_token, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DFLASH_H_ */

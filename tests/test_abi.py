@@ -1,0 +1,71 @@
+"""The C-ABI library: it loads, exports every declared symbol, and rejects bad
+arguments on the host before touching the GPU (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dflash.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dflash_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_draft_selection_b200 import build
+    build.build_library()
+    return ctypes.CDLL(build.LIB)
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert len(names) >= 7
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    lib.dflash_status_string.restype = ctypes.c_char_p
+    seen = set()
+    for code in range(7):
+        s = lib.dflash_status_string(code).decode()
+        assert s and s != "unknown status"
+        seen.add(s)
+    assert len(seen) == 7
+    assert lib.dflash_status_string(99).decode() == "unknown status"
+
+
+def test_host_side_rejections(lib):
+    vp = ctypes.c_void_p
+    fake = vp(0x1000)  # never dereferenced: every call below fails validation first
+    # K != 16
+    r = lib.dflash_lmhead_topk(fake, fake, 4, 4096, 256, 15, fake, fake, None, fake, ctypes.c_size_t(1 << 20),
+                               None, None)
+    assert r == 1
+    # null H
+    r = lib.dflash_lmhead_topk(None, fake, 4, 4096, 256, 16, fake, fake, None, fake, ctypes.c_size_t(1 << 20),
+                               None, None)
+    assert r == 1
+    # conv: d not a multiple of 8, null x
+    assert lib.dflash_conv2tap(fake, None, fake, fake, fake, 1, 5, 12, None) == 1
+    assert lib.dflash_conv2tap(None, None, fake, fake, fake, 1, 5, 16, None) == 1
+    # select: r not a multiple of 8, L > 16, K != 16
+    assert lib.dflash_path_select(fake, fake, fake, fake, 1, 4, 16, 12, 100, fake, None, None, None, None, None) == 1
+    assert lib.dflash_path_select(fake, fake, fake, fake, 1, 17, 16, 32, 100, fake, None, None, None, None, None) == 1
+    assert lib.dflash_path_select(fake, fake, fake, fake, 1, 4, 8, 32, 100, fake, None, None, None, None, None) == 1
+    # verify: L out of range
+    assert lib.dflash_verify(fake, fake, 1, 0, fake, fake, None) == 1
+    assert lib.dflash_verify(fake, fake, 1, 33, fake, fake, None) == 1
+
+
+def test_workspace_rejects_bad_sizes(lib):
+    lib.dflash_lmhead_topk_workspace.restype = ctypes.c_size_t
+    assert lib.dflash_lmhead_topk_workspace(0, 4096, 256) == 0
+    assert lib.dflash_lmhead_topk_workspace(4, 8, 256) == 0
+    assert lib.dflash_lmhead_topk_workspace(4, 4096, 100) == 0

@@ -1,0 +1,489 @@
+#!/usr/bin/env python
+"""Draft blocks/s of one draft cycle on B200: conv2tap + LM-head top-16 +
+path selection + verification.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one pass of the whole path over one batch of B blocks: the two-tap
+conv on [B, P, d], the fused LM head + log-softmax + top-16 on [B*L, d] x
+[V, d], pair scores + max-sum walk, greedy verification against the target's
+tokens.  Inputs are seeded synthetic arrays of the workload's shapes and
+distributions (block_draft_synth); W alone is larger than L2, so steps do not
+reuse each other's data through L2.
+
+Multi-GPU: one process per GPU (torchrun); blocks are independent, so each
+rank runs its own batch with replicated weights and no data-path collective
+(weak scaling).  The timed region is bracketed by a barrier and a device
+synchronize; the elapsed device time is the max over ranks.
+
+`--impl reference` times the CPU oracle (float64 numpy) on the host's cores on
+a bounded sample of the same workload; it is a deliberately slow baseline.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import block_draft_synth as syn  # noqa: E402
+
+METRIC = "draft blocks/sec (LM-head+top16+select+verify) on 1 B200; % of roofline"
+UNIT = "blocks/s"
+DEFAULT_WORKLOAD = "qwen3-4b-bs1"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# ------------------------------------------------------------------ helpers --
+
+def dist_env():
+    """(rank, local_rank, world_size) from the torchrun environment."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def rank_workload(w: syn.Workload, rank: int) -> syn.Workload:
+    """Per-rank batch: the same weights, different blocks (hidden states,
+    targets, conv inputs are drawn from a rank-specific seed)."""
+    import dataclasses
+    return w if rank == 0 else dataclasses.replace(w, seed=w.seed + 7919 * rank)
+
+
+def reduce_max(value: float, world: int) -> float:
+    """Max of a host float over all ranks (plumbing, not the data path)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(blocks_per_rank: int, world: int, ms_max: float, steps: int) -> float:
+    """Whole-job blocks/s: blocks all ranks processed / the slowest rank's time."""
+    return blocks_per_rank * world * steps / (ms_max / 1e3)
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": FALLBACK_BF16_TFLOPS}, "fallback"
+
+
+def lmhead_algorithmic(w: syn.Workload):
+    """Algorithmic bytes and FLOPs of one LM-head top-16 launch: W and H read
+    once, the candidate lists and lse written once; 2*M*d*V FLOPs."""
+    bytes_ = 2 * w.V * w.d + 2 * w.M * w.d + w.M * (16 * 8 + 4)
+    flops = 2.0 * w.M * w.d * w.V
+    return bytes_, flops
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for name in ("lmhead_topk.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "block_draft_selection_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the LM-head kernel from the committed ncu
+    summary for this workload, if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", f"lmhead_topk_{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    vals = {}
+    for line in text.splitlines():
+        if line.startswith("- ") and ":" in line:
+            k, v = line[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch_full_workload"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
+               0x1: "gpu_idle"}
+
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], set()
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _sample(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        for bit, name in self.REASONS.items():
+            if mask & bit and name != "gpu_idle":
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._sample()
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+            try:
+                self._sample()
+            except Exception:
+                pass
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------- GPU arm ----
+
+class Step:
+    """One draft cycle on device-resident buffers, through the C ABI."""
+
+    def __init__(self, w: syn.Workload, rank: int, device):
+        import torch
+        import block_draft_selection_b200 as bds
+        self.bds, self.torch, self.w = bds, torch, w
+        wr = rank_workload(w, rank)
+        dev = device
+        self.W = bds.bf16_tensor(syn.lm_head(w), dev)
+        E, M = syn.selector_tables(w)
+        self.E, self.Msel = bds.bf16_tensor(E, dev), bds.bf16_tensor(M, dev)
+        a0, a1 = syn.conv_taps(w)
+        self.a0, self.a1 = bds.bf16_tensor(a0, dev), bds.bf16_tensor(a1, dev)
+        # per-step inputs, also kept in pinned host memory for the end-to-end leg
+        H = syn.hidden(wr)
+        x, prev = syn.conv_input(wr)
+        self.H = bds.bf16_tensor(H, dev)
+        self.x, self.prev = bds.bf16_tensor(x, dev), bds.bf16_tensor(prev, dev)
+        # target tokens: the greedy choice of the same head on the noised hidden
+        # states (computed once with the library's own LM head, outside timing)
+        Hn = bds.bf16_tensor(syn.target_hidden(wr, H), dev)
+        _, tix, _ = bds.dflash_lmhead_topk(Hn, self.W)
+        self.target = tix[:, 0].contiguous().view(w.B, w.L + 1)
+        # outputs and workspace, allocated once
+        self.ws = bds.workspace(w.M, w.V, w.d, dev)
+        self.y = torch.empty_like(self.x)
+        self.lp = torch.empty((w.M, 16), dtype=torch.float32, device=dev)
+        self.ix = torch.empty((w.M, 16), dtype=torch.int32, device=dev)
+        self.lse = torch.empty(w.M, dtype=torch.float32, device=dev)
+        self.tok = torch.empty((w.B, w.L), dtype=torch.int32, device=dev)
+        self.slot = torch.empty((w.B, w.L), dtype=torch.int32, device=dev)
+        self.score = torch.empty(w.B, dtype=torch.float32, device=dev)
+        self.acc = torch.empty(w.B, dtype=torch.int32, device=dev)
+        self.nxt = torch.empty(w.B, dtype=torch.int32, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        # pinned host copies for the end-to-end leg
+        pin = lambda t: t.cpu().pin_memory()
+        self.h_in = [pin(self.H), pin(self.x), pin(self.prev), pin(self.target)]
+        self.h_out = [torch.empty_like(t, device="cpu").pin_memory()
+                      for t in (self.tok, self.acc, self.nxt, self.y)]
+
+    LAUNCHES_PER_STEP = 5   # conv, LM-head GEMM+epilogue, LM-head merge, select, verify
+
+    def run(self, ev=None):
+        bds = self.bds
+        bds.dflash_conv2tap(self.x, self.a0, self.a1, self.prev, y=self.y)
+        if ev is not None:
+            ev[0].record()
+        bds.dflash_lmhead_topk(self.H, self.W, topk_logp=self.lp, topk_idx=self.ix, lse=self.lse,
+                               ws=self.ws, dev_status=self.status)
+        if ev is not None:
+            ev[1].record()
+        bds.dflash_path_select(self.lp, self.ix, self.E, self.Msel, self.w.B, self.w.L,
+                               path_tok=self.tok, path_slot=self.slot, path_score=self.score)
+        bds.dflash_verify(self.tok, self.target, accept_len=self.acc, next_token=self.nxt)
+
+    def run_e2e(self):
+        """Host buffers in, host buffers out: H2D of the step's inputs, the
+        cycle, D2H of its results; the host reads the result (synchronize)."""
+        for dst, src in zip((self.H, self.x, self.prev, self.target), self.h_in):
+            dst.copy_(src, non_blocking=True)
+        self.run()
+        for dst, src in zip(self.h_out, (self.tok, self.acc, self.nxt, self.y)):
+            dst.copy_(src, non_blocking=True)
+        self.torch.cuda.current_stream().synchronize()
+
+    def io_bytes(self):
+        nb = lambda ts: int(sum(t.numel() * t.element_size() for t in ts))
+        return nb(self.h_in), nb(self.h_out)
+
+
+def gpu_arm(args, w: syn.Workload):
+    import torch
+    rank, local_rank, world = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=torch.device("cuda", local_rank))
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    step = Step(w, rank, device)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step.run()
+    barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    lm_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.steps)]
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        t0.record()
+        for k in range(args.steps):
+            step.run(lm_ev[k])
+        t1.record()
+        torch.cuda.synchronize()
+    barrier()
+    if int(step.status.item()) != 0:
+        raise RuntimeError(f"device status {int(step.status.item())} during the timed region")
+    ms = t0.elapsed_time(t1)
+    lm_ms = statistics.mean(a.elapsed_time(b) for a, b in lm_ev)
+    ms_max = reduce_max(ms, world)
+    value = aggregate(w.B, world, ms_max, args.steps)
+
+    # end-to-end leg: pinned host inputs -> device -> cycle -> host results
+    for _ in range(max(1, args.warmup // 2)):
+        step.run_e2e()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_steps = max(1, args.steps)
+    e0.record()
+    for _ in range(e_steps):
+        step.run_e2e()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    e_ms = reduce_max(e0.elapsed_time(e1), world)
+    h2d, d2h = step.io_bytes()
+
+    peaks, peaks_kind = load_peaks()
+    alg_bytes, alg_flops = lmhead_algorithmic(w)
+    t_lm = lm_ms / 1e3
+    hbm_t = alg_bytes / (peaks["hbm_gbs"] * 1e9)
+    tc_t = alg_flops / (peaks["bf16_tflops"] * 1e12)
+    if hbm_t >= tc_t:
+        roof = {"bound": "hbm", "achieved": alg_bytes / t_lm / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        pk = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        roof = {"bound": "tensor", "achieved": alg_flops / t_lm / 1e12, "peak": pk, "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = profiled_traffic(w.name)
+    roof["peak_source"] = peaks_kind
+    roof["kernel"] = "dflash_lmhead_topk (GEMM+epilogue and merge kernels)"
+    roof["algorithmic_per_launch"] = alg_bytes if roof["bound"] == "hbm" else alg_flops
+    roof["launch_ms"] = lm_ms
+
+    out = None
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded block_draft_synth; random-init weights of the workload's shapes)",
+            "config": {"workload": w.name, "blocks_per_gpu": w.B, "L": w.L, "M": w.M, "d": w.d, "V": w.V,
+                       "K": 16, "r": w.r, "conv": [w.B, w.P, w.d], "parallelism": f"dp{world} (blocks)",
+                       "l2": "inputs larger than L2 (W is %.0f MB > 126 MB)" % (2 * w.V * w.d / 1e6)},
+            "e2e": {"value": aggregate(w.B, world, e_ms, e_steps), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": Step.LAUNCHES_PER_STEP * args.steps,
+            "roofline": roof,
+            "clocks": clk.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return out
+
+
+# --------------------------------------------------------------- CPU oracle --
+
+class OracleSample:
+    """The CPU oracle, as it stands, on a bounded sample of the workload.
+
+    One sample step runs the oracle's conv on the full conv input, its LM head
+    + top-16 on a slice of the vocabulary (rows [v0, v0+Vs) of W, rotating
+    over steps), and its path selection + verification on the slice's lists.
+    The LM-head part is the only one whose work depends on V, and it grows in
+    proportion to V, so a full cycle is estimated as
+    t_cycle = (V / Vs) * t_lmhead_slice + t_rest."""
+
+    def __init__(self, w: syn.Workload):
+        import oracle
+        self.o, self.w = oracle, w
+        self.H, self.W = syn.hidden(w), syn.lm_head(w)
+        self.E, self.M = syn.selector_tables(w)
+        self.x, self.prev = syn.conv_input(w)
+        self.a0, self.a1 = syn.conv_taps(w)
+        self.target = np.random.default_rng(0).integers(0, w.V, size=(w.B, w.L + 1))
+        self.v0 = 0
+
+    def step(self, Vs: int):
+        o, w = self.o, self.w
+        Vs = max(16, min(Vs, w.V))
+        if self.v0 + Vs > w.V:
+            self.v0 = 0
+        sl = slice(self.v0, self.v0 + Vs)
+        self.v0 += Vs
+        t0 = time.perf_counter()
+        lp, ix, _ = o.lmhead_topk(self.H, self.W[sl], 16)
+        t1 = time.perf_counter()
+        o.conv2tap(self.x, self.prev, self.a0, self.a1)
+        sel = o.path_select(lp, ix, self.E[sl], self.M, w.B, w.L)
+        o.verify(sel["path_tok"], self.target)
+        t2 = time.perf_counter()
+        return t1 - t0, t2 - t1, Vs
+
+    def estimate(self, recs):
+        """blocks/s from recorded (t_lm, t_rest, Vs) steps."""
+        w = self.w
+        t_cycle = statistics.mean(t_lm * (w.V / vs) for t_lm, _, vs in recs) + statistics.mean(r for _, r, _ in recs)
+        return w.B / t_cycle, t_cycle
+
+
+def _threads_used():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+def _size_slice(smp: OracleSample, per_step_s: float) -> int:
+    """Vocabulary slice whose sample step takes about per_step_s seconds."""
+    w = smp.w
+    Vs = min(w.V, 4096)
+    t_lm, t_rest, _ = smp.step(Vs)
+    per_row = t_lm / Vs
+    return int(max(256, min(w.V, (per_step_s - t_rest) / max(per_row, 1e-12))))
+
+
+def cpu_baseline(w: syn.Workload, seconds: float):
+    """The oracle timed for about `seconds` of host CPU work on a bounded sample."""
+    smp = OracleSample(w)
+    Vs = _size_slice(smp, per_step_s=max(0.05, seconds / 8))
+    recs, t_start = [], time.perf_counter()
+    while time.perf_counter() - t_start < seconds or len(recs) < 2:
+        recs.append(smp.step(Vs))
+    value, t_cycle = smp.estimate(recs)
+    return {"value": value, "unit": UNIT, "cores": _threads_used(), "kind": "oracle",
+            "sample": (f"{len(recs)} oracle steps on workload {w.name}: conv + selection + verification of "
+                       f"all {w.B} block(s) per step, LM head on a {Vs}-row vocabulary slice (of {w.V}); "
+                       f"cycle time estimated as (V/slice)*t_lmhead + t_rest = {t_cycle:.3f} s"),
+            "host_cores_available": len(os.sched_getaffinity(0))}
+
+
+def reference_arm(args, w: syn.Workload):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return None
+    smp = OracleSample(w)
+    budget = float(args.ref_budget_s)
+    Vs = _size_slice(smp, per_step_s=max(0.01, budget / (args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        smp.step(Vs)
+    recs = [smp.step(Vs) for _ in range(args.steps)]
+    value, t_cycle = smp.estimate(recs)
+    cb = {"value": value, "unit": UNIT, "cores": _threads_used(), "kind": "oracle",
+          "sample": (f"each step: oracle conv + selection + verification of all {w.B} block(s), LM head on a "
+                     f"{Vs}-row slice of the {w.V}-row vocabulary; blocks/s from "
+                     f"(V/slice)*t_lmhead + t_rest = {t_cycle:.3f} s per cycle"),
+          "host_cores_available": len(os.sched_getaffinity(0))}
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_cycle,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded block_draft_synth)",
+            "config": {"workload": w.name, "blocks_per_gpu": w.B, "L": w.L, "M": w.M, "d": w.d, "V": w.V,
+                       "K": 16, "r": w.r, "conv": [w.B, w.P, w.d], "parallelism": "host cores"},
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=[x.name for x in syn.WORKLOADS])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-budget-s", type=float, default=120.0,
+                    help="host seconds the --impl reference run aims to take")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    w = syn.workload(args.workload)
+    if args.impl == "reference":
+        out = reference_arm(args, w)
+    else:
+        out = gpu_arm(args, w)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

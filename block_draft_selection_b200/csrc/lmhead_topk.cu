@@ -650,3 +650,67 @@ extern "C" int dflash_lmhead_logits_debug(const dflash_bf16* H, const dflash_bf1
   if (!z) return DFLASH_ERR_INVALID_ARG;
   return dflash::lm::launch(H, W, M, V, d, nullptr, nullptr, nullptr, z, ws, ws_bytes, dev_status, stream);
 }
+
+// ---------------------------------------------------------------------------
+// No-allocation variant of dflash_lmhead_topk.
+//
+// Some callers cannot hand this library a device workspace: code running
+// inside a custom allocator's own callbacks, engines whose memory pool is
+// fully reserved up front, and hosts that forbid cudaMalloc after start-up
+// (for example while other work is being captured or replayed).  For them,
+// the per-row partial records live in the file-scope array below instead of
+// a caller buffer.  The array is part of the library image: every GPU that
+// loads libdflash.so holds DFLASH_STATIC_SCRATCH_BYTES of it until the
+// process exits.
+//
+// Host code cannot use `g_static_scratch` as a pointer (its host-side name is
+// only a stand-in for the device symbol), so the device address is looked up
+// with cudaGetSymbolAddress once per device, with that device current, on the
+// first call made while it is current.  That first call on a device should
+// therefore happen before any stream capture begins.
+//
+// Every call shares the one array: calls that can overlap on the GPU (other
+// streams, other host threads on the same device) race on it and must be
+// serialised by the caller.  Nothing in it needs clearing between calls:
+// every record the merge step reads is written earlier in the same call.
+// ---------------------------------------------------------------------------
+
+static __device__ __align__(256) unsigned char g_static_scratch[DFLASH_STATIC_SCRATCH_BYTES];
+
+namespace dflash {
+namespace lm {
+
+constexpr int kMaxDevices = 64;
+static std::mutex g_static_mu;
+static void* g_static_ptr[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device (looked up once).
+static int static_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DFLASH_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (g_static_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return DFLASH_ERR_CUDA;
+    g_static_ptr[dev] = p;
+  }
+  *out = g_static_ptr[dev];
+  return DFLASH_OK;
+}
+
+}  // namespace lm
+}  // namespace dflash
+
+extern "C" int dflash_lmhead_topk_static(const dflash_bf16* H, const dflash_bf16* W, int M, int V, int d, int K,
+                                         float* topk_logp, int32_t* topk_idx, float* lse, int* dev_status,
+                                         void* stream) {
+  if (K != dflash::KTOP || !topk_logp || !topk_idx || !H || !W) return DFLASH_ERR_INVALID_ARG;
+  const size_t need = dflash_lmhead_topk_workspace(M, V, d);
+  if (need == 0) return DFLASH_ERR_INVALID_ARG;
+  if (need > static_cast<size_t>(DFLASH_STATIC_SCRATCH_BYTES)) return DFLASH_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  const int rc = dflash::lm::static_scratch(&scratch);
+  if (rc != DFLASH_OK) return rc;
+  return dflash::lm::launch(H, W, M, V, d, topk_logp, topk_idx, lse, nullptr, scratch,
+                            static_cast<size_t>(DFLASH_STATIC_SCRATCH_BYTES), dev_status, stream);
+}

@@ -101,6 +101,31 @@ int dflash_lmhead_topk(const dflash_bf16* H, const dflash_bf16* W, int M, int V,
                        float* topk_logp, int32_t* topk_idx, float* lse, void* ws, size_t ws_bytes,
                        int* dev_status, void* stream);
 
+/* Size of the library-owned scratch array used by dflash_lmhead_topk_static. */
+#define DFLASH_STATIC_SCRATCH_BYTES (8u << 20)
+
+/*
+ * dflash_lmhead_topk without a caller workspace.  The paper has no
+ * counterpart to this entry point.  For callers that cannot
+ * allocate device memory when they call, e.g. code inside an allocator's own
+ * hooks or engines whose device memory is all reserved up front.  Same inputs,
+ * outputs and results as dflash_lmhead_topk; the partial records go to a
+ * library-owned device array of DFLASH_STATIC_SCRATCH_BYTES (8 MiB), which
+ * every GPU that loads the library holds until the process exits.
+ *
+ * Limit: dflash_lmhead_topk_workspace(M, V, d) must not exceed
+ * DFLASH_STATIC_SCRATCH_BYTES, else the call returns DFLASH_ERR_UNSUPPORTED
+ * (M <= 128 at V = 151,936 fits; large-M shapes generally do not).
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current, so make that first call
+ * before any stream capture.  Calls share the array: calls that may overlap
+ * on the GPU (different streams or threads on one device) race and must be
+ * serialised by the caller.  The call allocates no memory.
+ */
+int dflash_lmhead_topk_static(const dflash_bf16* H, const dflash_bf16* W, int M, int V, int d, int K,
+                              float* topk_logp, int32_t* topk_idx, float* lse, int* dev_status,
+                              void* stream);
+
 /*
  * Diagnostic: the same GEMM path as dflash_lmhead_topk, but writing the raw
  * logits z [M, V] fp32 (row-major) instead of selecting.  Meant for small

@@ -233,17 +233,20 @@ class Step:
     LAUNCHES_PER_STEP = 5   # conv, LM-head GEMM+epilogue, LM-head merge, select, verify
 
     def run(self, ev=None):
+        """One cycle.  `ev`: optional 5 CUDA events recorded between the stages."""
         bds = self.bds
+        rec = (lambda k: ev[k].record()) if ev is not None else (lambda k: None)
+        rec(0)
         bds.dflash_conv2tap(self.x, self.a0, self.a1, self.prev, y=self.y)
-        if ev is not None:
-            ev[0].record()
+        rec(1)
         bds.dflash_lmhead_topk(self.H, self.W, topk_logp=self.lp, topk_idx=self.ix, lse=self.lse,
                                ws=self.ws, dev_status=self.status)
-        if ev is not None:
-            ev[1].record()
+        rec(2)
         bds.dflash_path_select(self.lp, self.ix, self.E, self.Msel, self.w.B, self.w.L,
                                path_tok=self.tok, path_slot=self.slot, path_score=self.score)
+        rec(3)
         bds.dflash_verify(self.tok, self.target, accept_len=self.acc, next_token=self.nxt)
+        rec(4)
 
     def run_e2e(self):
         """Host buffers in, host buffers out: H2D of the step's inputs, the
@@ -284,19 +287,19 @@ def gpu_arm(args, w: syn.Workload):
         step.run()
     barrier()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    lm_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-             for _ in range(args.steps)]
+    st_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     with ClockSampler(device.index if device.index is not None else 0) as clk:
         t0.record()
         for k in range(args.steps):
-            step.run(lm_ev[k])
+            step.run(st_ev[k])
         t1.record()
         torch.cuda.synchronize()
     barrier()
     if int(step.status.item()) != 0:
         raise RuntimeError(f"device status {int(step.status.item())} during the timed region")
     ms = t0.elapsed_time(t1)
-    lm_ms = statistics.mean(a.elapsed_time(b) for a, b in lm_ev)
+    stage_ms = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in st_ev) for j in range(4)]
+    lm_ms = stage_ms[1]
     ms_max = reduce_max(ms, world)
     value = aggregate(w.B, world, ms_max, args.steps)
 
@@ -346,6 +349,9 @@ def gpu_arm(args, w: syn.Workload):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": Step.LAUNCHES_PER_STEP * args.steps,
             "roofline": roof,
+            "stages_us": {"conv2tap": 1e3 * stage_ms[0], "lmhead_topk": 1e3 * stage_ms[1],
+                          "path_select": 1e3 * stage_ms[2], "verify": 1e3 * stage_ms[3],
+                          "select_plus_verify_share": (stage_ms[2] + stage_ms[3]) / (ms_max / args.steps)},
             "clocks": clk.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:

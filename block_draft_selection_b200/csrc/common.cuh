@@ -246,19 +246,36 @@ struct TopState {
   }
 
   // Insert (x, ix) if it beats the current 16th entry under the full order.
+  // The list is sorted, so the entries that stay ahead of x form a prefix;
+  // every slot's new content depends only on two compares of the old list,
+  // so the 16 slots update in parallel (no serial bubble chain).
   __device__ __forceinline__ void insert(float x, int ix) {
     if (!better(x, ix, v[KTOP - 1], i[KTOP - 1])) return;
-    v[KTOP - 1] = x;
-    i[KTOP - 1] = ix;
+    bool ahead[KTOP];
 #pragma unroll
-    for (int k = KTOP - 1; k > 0; --k) {
-      const bool sw = better(v[k], i[k], v[k - 1], i[k - 1]);
-      const float a = v[k], b = v[k - 1];
-      const int ia = i[k], ib = i[k - 1];
-      v[k - 1] = sw ? a : b;
-      v[k] = sw ? b : a;
-      i[k - 1] = sw ? ia : ib;
-      i[k] = sw ? ib : ia;
+    for (int k = 0; k < KTOP; ++k) ahead[k] = better(v[k], i[k], x, ix);
+    float nv[KTOP];
+    int ni[KTOP];
+    nv[0] = ahead[0] ? v[0] : x;
+    ni[0] = ahead[0] ? i[0] : ix;
+#pragma unroll
+    for (int k = 1; k < KTOP; ++k) {
+      nv[k] = ahead[k] ? v[k] : (ahead[k - 1] ? x : v[k - 1]);
+      ni[k] = ahead[k] ? i[k] : (ahead[k - 1] ? ix : i[k - 1]);
+    }
+#pragma unroll
+    for (int k = 0; k < KTOP; ++k) {
+      v[k] = nv[k];
+      i[k] = ni[k];
+    }
+  }
+
+  // Insert the entries of another sorted list while they beat the 16th entry.
+  __device__ __forceinline__ void insert_sorted(const float (&ov)[KTOP], const int (&oi)[KTOP]) {
+#pragma unroll
+    for (int k = 0; k < KTOP; ++k) {
+      if (!better(ov[k], oi[k], v[KTOP - 1], i[KTOP - 1])) break;
+      insert(ov[k], oi[k]);
     }
   }
 
@@ -297,5 +314,43 @@ struct __align__(16) Partial {
   int i[KTOP];
 };
 static_assert(sizeof(Partial) == 144, "partial record layout");
+
+// Store a list as one partial record with 16-byte stores.
+__device__ __forceinline__ void store_partial(Partial* rec, float m, float s, const float (&v)[KTOP],
+                                              const int (&i)[KTOP]) {
+  float4* d = reinterpret_cast<float4*>(rec);
+  d[0] = make_float4(m, s, 0.f, 0.f);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) d[1 + q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    d[5 + q] = make_float4(__int_as_float(i[4 * q]), __int_as_float(i[4 * q + 1]), __int_as_float(i[4 * q + 2]),
+                           __int_as_float(i[4 * q + 3]));
+}
+
+// Load a partial record with 16-byte read-only loads.
+struct PartialRegs {
+  float4 q[9];
+  __device__ __forceinline__ void load(const Partial* rec) {
+    const float4* s = reinterpret_cast<const float4*>(rec);
+#pragma unroll
+    for (int k = 0; k < 9; ++k) q[k] = __ldg(s + k);
+  }
+  __device__ __forceinline__ float m() const { return q[0].x; }
+  __device__ __forceinline__ float s() const { return q[0].y; }
+  __device__ __forceinline__ void lists(float (&v)[KTOP], int (&i)[KTOP]) const {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[4 * k] = q[1 + k].x;
+      v[4 * k + 1] = q[1 + k].y;
+      v[4 * k + 2] = q[1 + k].z;
+      v[4 * k + 3] = q[1 + k].w;
+      i[4 * k] = __float_as_int(q[5 + k].x);
+      i[4 * k + 1] = __float_as_int(q[5 + k].y);
+      i[4 * k + 2] = __float_as_int(q[5 + k].z);
+      i[4 * k + 3] = __float_as_int(q[5 + k].w);
+    }
+  }
+};
 
 }  // namespace dflash

@@ -47,6 +47,15 @@ constexpr int EPI_THREADS = 128;
 constexpr int SMEM_BUDGET = 224 * 1024;
 
 enum { MODE_SWAP = 0, MODE_LARGE = 1 };
+// LARGE-orientation tile schedules:
+//  STRIDED  tile t = cta + k * grid in vocabulary-major order: the CTAs running
+//           at one time cover a narrow vocabulary window (W tiles are shared
+//           through L2); each tile starts a fresh candidate list.
+//  RUNS     CTA c owns m-tile (c % m_tiles) over one contiguous vocabulary range
+//           (range c / m_tiles of nr); the CTAs owning one range walk it in
+//           lockstep (W shared through L2) and each keeps its candidate list
+//           across the whole range, so few values reach the insertion code.
+enum { SCHED_STRIDED = 0, SCHED_RUNS = 1 };
 
 struct Params {
   int M, V, d;
@@ -64,6 +73,8 @@ struct Params {
   int t_bytes;
   // LARGE
   int m_tiles, v_tiles;
+  int sched;         // SCHED_STRIDED or SCHED_RUNS
+  int nr;            // SCHED_RUNS: vocabulary ranges per m-tile
   // outputs
   Partial* part;     // [M][P]
   int P;
@@ -95,6 +106,32 @@ __device__ __forceinline__ void swap_range(const Params& p, int& r0, int& r1) {
   const long long c = blockIdx.x;
   r0 = static_cast<int>((c * p.units) / G) * 16;
   r1 = static_cast<int>(((c + 1) * p.units) / G) * 16;
+}
+
+// LARGE: the k-th tile of this CTA; false past the end.  `slot` names the
+// partial record the tile's run writes; first/last mark the run's ends.
+__device__ __forceinline__ bool large_tile(const Params& p, int k, int& mt, int& vt, int& slot, bool& first,
+                                           bool& last) {
+  if (p.sched == SCHED_RUNS) {
+    const int c = blockIdx.x;
+    mt = c % p.m_tiles;
+    const int r = c / p.m_tiles;
+    const int lo = static_cast<int>(static_cast<long long>(r) * p.v_tiles / p.nr);
+    const int hi = static_cast<int>(static_cast<long long>(r + 1) * p.v_tiles / p.nr);
+    vt = lo + k;
+    if (vt >= hi) return false;
+    slot = r;
+    first = k == 0;
+    last = vt == hi - 1;
+    return true;
+  }
+  const long long t = blockIdx.x + static_cast<long long>(k) * gridDim.x;
+  if (t >= static_cast<long long>(p.m_tiles) * p.v_tiles) return false;
+  vt = static_cast<int>(t / p.m_tiles);
+  mt = static_cast<int>(t - static_cast<long long>(vt) * p.m_tiles);
+  slot = vt;
+  first = last = true;
+  return true;
 }
 
 // ------------------------------------------------------------ kernel -------
@@ -149,7 +186,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   int r0 = 0, r1 = 0;
   if (MODE == MODE_SWAP) swap_range(p, r0, r1);
-  const int num_tiles_large = p.m_tiles * p.v_tiles;
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
@@ -184,9 +220,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       } else {
-        for (int t = blockIdx.x; ok && t < num_tiles_large; t += gridDim.x) {
-          const int vt = t / p.m_tiles;
-          const int mt = t - vt * p.m_tiles;
+        int mt, vt, slot;
+        bool first, last;
+        for (int k = 0; ok && large_tile(p, k, mt, vt, slot, first, last); ++k) {
           for (int kc = 0; kc < p.num_kc; ++kc) {
             if (!mbar_wait(empty_bar(s), ph ^ 1u, deadline, abort_flag, p.status)) {
               ok = false;
@@ -248,7 +284,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (MODE == MODE_SWAP) {
         for (int t0 = r0; ok && t0 < r1; t0 += A_ROWS) ok = do_tile();
       } else {
-        for (int t = blockIdx.x; ok && t < num_tiles_large; t += gridDim.x) ok = do_tile();
+        int mt, vt, slot;
+        bool first, last;
+        for (int k = 0; ok && large_tile(p, k, mt, vt, slot, first, last); ++k) ok = do_tile();
       }
       // Every MMA this thread issued has completed before TMEM is released.
       umma_commit(drain_bar);
@@ -334,26 +372,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ov[r] = bv;
         oi[r] = bi;
       }
-      if (active && sub == 0) {
-        Partial* rec = p.part + static_cast<size_t>(n) * p.P + blockIdx.x;
-        rec->m = st.m;
-        rec->s = st.s;
-#pragma unroll
-        for (int r = 0; r < KTOP; ++r) {
-          rec->v[r] = ov[r];
-          rec->i[r] = oi[r];
-        }
-      }
+      if (active && sub == 0) store_partial(p.part + static_cast<size_t>(n) * p.P + blockIdx.x, st.m, st.s, ov, oi);
     } else {
-      for (int t = blockIdx.x; t < num_tiles_large; t += gridDim.x) {
-        const int vt = t / p.m_tiles;
-        const int mt = t - vt * p.m_tiles;
+      int mt, vt, slot;
+      bool first, last;
+      for (int k = 0; large_tile(p, k, mt, vt, slot, first, last); ++k) {
         int ok = 0;
         if (lane == 0) ok = mbar_wait(tfull_bar(tb), tph, deadline, abort_flag, p.status) ? 1 : 0;
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         tc_fence_after();
-        st.reset();
+        if (first) st.reset();
         const int row = mt * A_ROWS + trow;
         const int v0 = vt * LARGE_N;
         const uint32_t taddr = tmem_base + static_cast<uint32_t>(tb * p.buf_cols) + lane_off;
@@ -371,10 +400,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             st.m = cmax;
           }
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            if (jj < nvalid) {
-              st.s += __expf(x[jj] - st.m);
-              st.insert(x[jj], v0 + c0 + jj);
+          for (int jj = 0; jj < 16; ++jj)
+            if (jj < nvalid) st.s += __expf(x[jj] - st.m);
+          // Candidates of this chunk that can enter the list; each lane then
+          // inserts only its own, so the warp loops max_lane(count) times.
+          uint32_t pend = 0;
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj)
+            if (jj < nvalid && x[jj] >= st.v[KTOP - 1]) pend |= 1u << jj;
+          while (__any_sync(0xffffffffu, pend != 0)) {
+            if (pend) {
+              const int jj = __ffs(pend) - 1;
+              pend &= pend - 1;
+              float xv = x[0];
+#pragma unroll
+              for (int q = 1; q < 16; ++q) xv = jj == q ? x[q] : xv;
+              st.insert(xv, v0 + c0 + jj);
             }
           }
           if (p.z_dbg && row < p.M) {
@@ -386,16 +427,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_before();
         mbar_arrive(tempty_bar(tb));
         if (++tb == 2) { tb = 0; tph ^= 1u; }
-        if (row < p.M) {
-          Partial* rec = p.part + static_cast<size_t>(row) * p.P + vt;
-          rec->m = st.m;
-          rec->s = st.s;
-#pragma unroll
-          for (int r = 0; r < KTOP; ++r) {
-            rec->v[r] = st.v[r];
-            rec->i[r] = st.i[r];
-          }
-        }
+        if (last && row < p.M) store_partial(p.part + static_cast<size_t>(row) * p.P + slot, st.m, st.s, st.v, st.i);
       }
     }
   }
@@ -420,16 +452,17 @@ __global__ void __launch_bounds__(128) merge_kernel(const Partial* __restrict__ 
   TopState st;
   st.reset();
   const Partial* base = part + static_cast<size_t>(row) * P;
+  // Records are loaded one ahead so the next load overlaps this record's work.
+  PartialRegs cur, nxt;
+  if (lane < P) cur.load(base + lane);
   for (int q = lane; q < P; q += 32) {
-    const Partial* rec = base + q;
-    st.merge_lse(rec->m, rec->s);
-#pragma unroll 1
-    for (int k = 0; k < KTOP; ++k) {
-      const float x = rec->v[k];
-      const int ix = rec->i[k];
-      if (!better(x, ix, st.v[KTOP - 1], st.i[KTOP - 1])) break;
-      st.insert(x, ix);
-    }
+    if (q + 32 < P) nxt.load(base + q + 32);
+    st.merge_lse(cur.m(), cur.s());
+    float rv[KTOP];
+    int ri[KTOP];
+    cur.lists(rv, ri);
+    st.insert_sorted(rv, ri);
+    cur = nxt;
   }
   for (int off = 1; off < 32; off <<= 1) {
     const float m2 = __shfl_xor_sync(0xffffffffu, st.m, off);
@@ -562,9 +595,23 @@ static bool make_plan(int M, int V, int d, int sms, Plan& pl) {
     p.t_bytes = 0;
     p.m_tiles = (M + A_ROWS - 1) / A_ROWS;
     p.v_tiles = (V + LARGE_N - 1) / LARGE_N;
-    const int tiles = p.m_tiles * p.v_tiles;
-    pl.grid = tiles < sms ? tiles : sms;
-    p.P = p.v_tiles;
+    const long long tiles = static_cast<long long>(p.m_tiles) * p.v_tiles;
+    const int g_str = static_cast<int>(tiles < sms ? tiles : sms);
+    const long long t_str = (tiles + g_str - 1) / g_str;           // tiles on the busiest CTA
+    int nr = sms / p.m_tiles;
+    if (nr > p.v_tiles) nr = p.v_tiles;
+    const long long t_run = nr >= 1 ? (p.v_tiles + nr - 1) / nr : (1ll << 40);
+    if (t_run <= t_str) {
+      p.sched = SCHED_RUNS;
+      p.nr = nr;
+      pl.grid = nr * p.m_tiles;
+      p.P = nr;
+    } else {
+      p.sched = SCHED_STRIDED;
+      p.nr = 0;
+      pl.grid = g_str;
+      p.P = p.v_tiles;
+    }
     p.stages = 4;
   }
   pl.smem = smem_layout(p).total + 1024;

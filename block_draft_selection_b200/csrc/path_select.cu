@@ -9,7 +9,7 @@
 // Walk: delta_0 = 0, delta_{i+1}[k] = max_j delta_i[j] + S_i[j,k] (ties: lowest
 // j), end at argmax_k delta_{L-1}[k] (ties: lowest k), then backtrack.
 //
-// One CTA (256 threads) per block:
+// One CTA per block (1024 threads when there are few blocks, else 256):
 //   1. gather the 16*L candidate rows of E and the matrix M into shared memory
 //      (bf16, rows padded by 16 bytes so 16-byte loads of 8 neighbouring rows
 //      hit distinct banks);
@@ -23,7 +23,7 @@
 namespace dflash {
 namespace sel {
 
-constexpr int THREADS = 256;
+constexpr int MAX_THREADS = 1024;
 constexpr int KC = 16;
 constexpr int U_BUDGET = 48 * 1024;
 
@@ -67,7 +67,7 @@ __host__ __device__ inline Layout layout(int L, int r) {
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-__global__ void __launch_bounds__(THREADS) path_select_kernel(
+__global__ void __launch_bounds__(MAX_THREADS) path_select_kernel(
     const float* __restrict__ topk_logp, const int32_t* __restrict__ topk_idx, const uint16_t* __restrict__ E,
     const uint16_t* __restrict__ Msel, int L, int r, int V, int32_t* __restrict__ path_tok,
     int32_t* __restrict__ path_slot, float* __restrict__ path_score, float* __restrict__ pair_dbg, int* status) {
@@ -83,11 +83,12 @@ __global__ void __launch_bounds__(THREADS) path_select_kernel(
 
   const int b = blockIdx.x;
   const int tid = threadIdx.x;
+  const int nthr = blockDim.x;
   const int r8 = r / 8;
   const size_t row0 = static_cast<size_t>(b) * L;
 
   // ---- 1. candidates, their E rows, and M into shared memory -------------
-  for (int q = tid; q < L * KC; q += THREADS) {
+  for (int q = tid; q < L * KC; q += nthr) {
     lps[q] = topk_logp[row0 * KC + q];
     int c = topk_idx[row0 * KC + q];
     if (c < 0 || c >= V) {
@@ -99,10 +100,10 @@ __global__ void __launch_bounds__(THREADS) path_select_kernel(
   {
     const uint4* Mg = reinterpret_cast<const uint4*>(Msel);
     uint4* Mv = reinterpret_cast<uint4*>(Ms);
-    for (int q = tid; q < r * r8; q += THREADS) Mv[q] = __ldg(Mg + q);
+    for (int q = tid; q < r * r8; q += nthr) Mv[q] = __ldg(Mg + q);
   }
   __syncthreads();
-  for (int q = tid; q < L * KC * r8; q += THREADS) {
+  for (int q = tid; q < L * KC * r8; q += nthr) {
     const int cand = q / r8;
     const int v8 = q - cand * r8;
     const uint4 val = __ldg(reinterpret_cast<const uint4*>(E + static_cast<size_t>(toks[cand]) * r) + v8);
@@ -115,7 +116,7 @@ __global__ void __launch_bounds__(THREADS) path_select_kernel(
   for (int i0 = 0; i0 < npos; i0 += lo.pc) {
     const int pcn = min(lo.pc, npos - i0);
     // u[ii][j][t] = sum_s e_{c_(i0+ii),j}[s] * M[s][t], 8 outputs per item
-    for (int q = tid; q < pcn * KC * r8; q += THREADS) {
+    for (int q = tid; q < pcn * KC * r8; q += nthr) {
       const int tg = q % r8;
       const int jj = q / r8;  // (ii * 16 + j)
       const int ii = jj / KC;
@@ -139,7 +140,7 @@ __global__ void __launch_bounds__(THREADS) path_select_kernel(
       *reinterpret_cast<float4*>(ur + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
     __syncthreads();
-    for (int q = tid; q < pcn * KC * KC; q += THREADS) {
+    for (int q = tid; q < pcn * KC * KC; q += nthr) {
       const int k = q % KC;
       const int j = (q / KC) % KC;
       const int ii = q / (KC * KC);
@@ -243,7 +244,10 @@ extern "C" int dflash_path_select(const float* topk_logp, const int32_t* topk_id
       return DFLASH_ERR_CUDA;
     attr_done = true;
   }
-  path_select_kernel<<<B, THREADS, lo.total, static_cast<cudaStream_t>(stream)>>>(
+  // Few blocks: spread each block's candidate work over more threads (latency);
+  // many blocks: 256 threads so several CTAs share an SM.
+  const int threads = B < 128 ? 1024 : 256;
+  path_select_kernel<<<B, threads, lo.total, static_cast<cudaStream_t>(stream)>>>(
       topk_logp, topk_idx, E, Msel, L, r, V, path_tok, path_slot, path_score, pair_scores_dbg, dev_status);
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }

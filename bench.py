@@ -202,7 +202,6 @@ class Step:
         self.E, self.Msel = bds.bf16_tensor(E, dev), bds.bf16_tensor(M, dev)
         a0, a1 = syn.conv_taps(w)
         self.a0, self.a1 = bds.bf16_tensor(a0, dev), bds.bf16_tensor(a1, dev)
-        # per-step inputs, also kept in pinned host memory for the end-to-end leg
         H = syn.hidden(wr)
         x, prev = syn.conv_input(wr)
         self.H = bds.bf16_tensor(H, dev)
@@ -212,59 +211,77 @@ class Step:
         Hn = bds.bf16_tensor(syn.target_hidden(wr, H), dev)
         _, tix, _ = bds.dflash_lmhead_topk(Hn, self.W)
         self.target = tix[:, 0].contiguous().view(w.B, w.L + 1)
-        # outputs and workspace, allocated once
         self.ws = bds.workspace(w.M, w.V, w.d, dev)
+        e = lambda shape, dt: torch.empty(shape, dtype=dt, device=dev)
         self.y = torch.empty_like(self.x)
-        self.lp = torch.empty((w.M, 16), dtype=torch.float32, device=dev)
-        self.ix = torch.empty((w.M, 16), dtype=torch.int32, device=dev)
-        self.lse = torch.empty(w.M, dtype=torch.float32, device=dev)
-        self.tok = torch.empty((w.B, w.L), dtype=torch.int32, device=dev)
-        self.slot = torch.empty((w.B, w.L), dtype=torch.int32, device=dev)
-        self.score = torch.empty(w.B, dtype=torch.float32, device=dev)
-        self.acc = torch.empty(w.B, dtype=torch.int32, device=dev)
-        self.nxt = torch.empty(w.B, dtype=torch.int32, device=dev)
+        self.lp, self.ix, self.lse = e((w.M, 16), torch.float32), e((w.M, 16), torch.int32), e(w.M, torch.float32)
+        self.tok, self.slot = e((w.B, w.L), torch.int32), e((w.B, w.L), torch.int32)
+        self.score, self.acc, self.nxt = e(w.B, torch.float32), e(w.B, torch.int32), e(w.B, torch.int32)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
-        # pinned host copies for the end-to-end leg
-        pin = lambda t: t.cpu().pin_memory()
-        self.h_in = [pin(self.H), pin(self.x), pin(self.prev), pin(self.target)]
-        self.h_out = [torch.empty_like(t, device="cpu").pin_memory()
-                      for t in (self.tok, self.acc, self.nxt, self.y)]
 
-    LAUNCHES_PER_STEP = 5   # conv, LM-head GEMM+epilogue, LM-head merge, select, verify
+    # conv, LM-head GEMM+epilogue, LM-head merge, select+verify
+    LAUNCHES_PER_STEP = 4
+    STAGES = ("conv2tap", "lmhead_topk", "select_verify")
+    TIMED = STAGES + ("event_pair",)
 
-    def run(self, ev=None):
-        """One cycle.  `ev`: optional 5 CUDA events recorded between the stages."""
+    def run(self, marks=None):
+        """One cycle.  `marks`: optional {stage name: (event, event)} recorded
+        around that stage's call."""
         bds = self.bds
-        rec = (lambda k: ev[k].record()) if ev is not None else (lambda k: None)
-        rec(0)
-        bds.dflash_conv2tap(self.x, self.a0, self.a1, self.prev, y=self.y)
-        rec(1)
-        bds.dflash_lmhead_topk(self.H, self.W, topk_logp=self.lp, topk_idx=self.ix, lse=self.lse,
-                               ws=self.ws, dev_status=self.status)
-        rec(2)
-        bds.dflash_path_select(self.lp, self.ix, self.E, self.Msel, self.w.B, self.w.L,
-                               path_tok=self.tok, path_slot=self.slot, path_score=self.score)
-        rec(3)
-        bds.dflash_verify(self.tok, self.target, accept_len=self.acc, next_token=self.nxt)
-        rec(4)
+        marks = marks or {}
 
-    def run_e2e(self):
-        """Host buffers in, host buffers out: H2D of the step's inputs, the
-        cycle, D2H of its results; the host reads the result (synchronize)."""
-        for dst, src in zip((self.H, self.x, self.prev, self.target), self.h_in):
-            dst.copy_(src, non_blocking=True)
-        self.run()
-        for dst, src in zip(self.h_out, (self.tok, self.acc, self.nxt, self.y)):
-            dst.copy_(src, non_blocking=True)
-        self.torch.cuda.current_stream().synchronize()
+        def stage(name, fn):
+            ev = marks.get(name)
+            if ev:
+                ev[0].record()
+            fn()
+            if ev:
+                ev[1].record()
 
-    def io_bytes(self):
-        nb = lambda ts: int(sum(t.numel() * t.element_size() for t in ts))
-        return nb(self.h_in), nb(self.h_out)
+        stage("event_pair", lambda: None)    # calibration: two event nodes, nothing between
+        stage("conv2tap", lambda: bds.dflash_conv2tap(self.x, self.a0, self.a1, self.prev, y=self.y))
+        stage("lmhead_topk", lambda: bds.dflash_lmhead_topk(
+            self.H, self.W, topk_logp=self.lp, topk_idx=self.ix, lse=self.lse, ws=self.ws, dev_status=self.status))
+        stage("select_verify", lambda: bds.dflash_select_verify(
+            self.lp, self.ix, self.E, self.Msel, self.target, self.w.B, self.w.L, path_tok=self.tok,
+            path_slot=self.slot, path_score=self.score, accept_len=self.acc, next_token=self.nxt,
+            dev_status=self.status))
+
+
+def _graph_steps(step, n_steps):
+    """Capture n_steps cycles into one CUDA graph.  Up to three of them carry
+    external timing events (event nodes) around one stage each -- the last
+    cycle around the LM head, the one before around select+verify, the one
+    before that around the conv -- so stage durations are sampled inside the
+    timed region at a cost of a few event nodes per graph."""
+    import torch
+    ev = lambda: (torch.cuda.Event(enable_timing=True, external=True),
+                  torch.cuda.Event(enable_timing=True, external=True))
+    plan = {n_steps - 1: "lmhead_topk", n_steps - 2: "select_verify", n_steps - 3: "conv2tap",
+            n_steps - 4: "event_pair"}
+    marks = {k: {name: ev()} for k, name in plan.items() if k >= 0}
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step.run()
+    side.synchronize()
+    with torch.cuda.graph(g, stream=side):
+        for k in range(n_steps):
+            step.run(marks.get(k))
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    return g, {name: pair for m in marks.values() for name, pair in m.items()}
+
+
+def _chunk(steps, cap=32):
+    """Largest divisor of `steps` not above `cap`: cycles per captured graph."""
+    return max(c for c in range(1, min(cap, steps) + 1) if steps % c == 0)
 
 
 def gpu_arm(args, w: syn.Workload):
     import torch
+    import block_draft_selection_b200 as bds
     rank, local_rank, world = dist_env()
     if world > 1:
         import datetime
@@ -285,38 +302,72 @@ def gpu_arm(args, w: syn.Workload):
 
     for _ in range(args.warmup):
         step.run()
-    barrier()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    st_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    samples = {n: [] for n in Step.TIMED}
+    if args.eager:
+        chunk, graphs = 1, []
+        marks = [{n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for n in Step.TIMED} for _ in range(args.steps)]
+    else:
+        chunk = _chunk(args.steps)
+        n_rep = args.steps // chunk
+        graphs = [_graph_steps(step, chunk) for _ in range(min(8, n_rep))]
+        for g, _ in graphs:
+            g.replay()              # one untimed replay of each captured graph
+    barrier()
     with ClockSampler(device.index if device.index is not None else 0) as clk:
         t0.record()
-        for k in range(args.steps):
-            step.run(st_ev[k])
+        if args.eager:
+            for k in range(args.steps):
+                step.run(marks[k])
+        else:
+            for rep in range(n_rep):
+                graphs[rep % len(graphs)][0].replay()
         t1.record()
         torch.cuda.synchronize()
     barrier()
     if int(step.status.item()) != 0:
         raise RuntimeError(f"device status {int(step.status.item())} during the timed region")
     ms = t0.elapsed_time(t1)
-    stage_ms = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in st_ev) for j in range(4)]
-    lm_ms = stage_ms[1]
+    # stage durations: every cycle of the eager loop, or the instrumented cycles
+    # of each graph's last replay inside the timed region
+    for m in (marks if args.eager else [gm for _, gm in graphs]):
+        for n, (a, b) in m.items():
+            samples[n].append(a.elapsed_time(b))
+    mean = lambda n: statistics.mean(samples[n]) if samples[n] else float("nan")
+    ev_ms = mean("event_pair") if samples["event_pair"] else 0.0
+    raw_ms = [mean(n) for n in Step.STAGES]
+    # net of the two event nodes that bracket each timed stage
+    stage_ms = [max(0.0, t - ev_ms) for t in raw_ms]
+    lm_ms = raw_ms[1]                   # gross: includes the bracketing event nodes (conservative)
+    lm_net_ms = stage_ms[1]
     ms_max = reduce_max(ms, world)
     value = aggregate(w.B, world, ms_max, args.steps)
+    del graphs
 
-    # end-to-end leg: pinned host inputs -> device -> cycle -> host results
-    for _ in range(max(1, args.warmup // 2)):
-        step.run_e2e()
+    # end-to-end leg: the library's DraftCycle, one graph launch per step that
+    # copies the step's inputs from pinned host memory, runs the cycle and
+    # copies the results back; the host waits for them every step
+    cyc = bds.DraftCycle(step.W, step.E, step.Msel, step.a0, step.a1, w.B, w.L, w.P)
+    cyc.host_in["H"].copy_(step.H)
+    cyc.host_in["x"].copy_(step.x)
+    cyc.host_in["prev"].copy_(step.prev)
+    cyc.host_in["target"].copy_(step.target)
+    for _ in range(max(3, args.warmup // 2)):
+        cyc.run()
     barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e_steps = max(1, args.steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(e_steps):
-        step.run_e2e()
+        cyc.run()
     e1.record()
     torch.cuda.synchronize()
     barrier()
+    if int(cyc.status.item()) != 0:
+        raise RuntimeError(f"device status {int(cyc.status.item())} in the end-to-end leg")
     e_ms = reduce_max(e0.elapsed_time(e1), world)
-    h2d, d2h = step.io_bytes()
+    h2d, d2h = cyc.io_bytes()
 
     peaks, peaks_kind = load_peaks()
     alg_bytes, alg_flops = lmhead_algorithmic(w)
@@ -329,11 +380,18 @@ def gpu_arm(args, w: syn.Workload):
         pk = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
         roof = {"bound": "tensor", "achieved": alg_flops / t_lm / 1e12, "peak": pk, "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
+    if roof["bound"] == "tensor":
+        # timed inside long runs of back-to-back cycles: the sustained peak is
+        # the denominator; the burst-peak fraction is given beside it
+        roof["peak_kind"] = "bf16_tflops_sustained"
+        roof["frac_of_burst"] = roof["achieved"] / peaks["bf16_tflops"]
     roof["traffic"] = profiled_traffic(w.name)
     roof["peak_source"] = peaks_kind
     roof["kernel"] = "dflash_lmhead_topk (GEMM+epilogue and merge kernels)"
     roof["algorithmic_per_launch"] = alg_bytes if roof["bound"] == "hbm" else alg_flops
     roof["launch_ms"] = lm_ms
+    roof["launch_ms_net_of_events"] = lm_net_ms
+    roof["frac_net_of_events"] = roof["frac"] * lm_ms / lm_net_ms if lm_net_ms > 0 else None
 
     out = None
     if rank == 0:
@@ -344,14 +402,19 @@ def gpu_arm(args, w: syn.Workload):
             "data": "synthetic (seeded block_draft_synth; random-init weights of the workload's shapes)",
             "config": {"workload": w.name, "blocks_per_gpu": w.B, "L": w.L, "M": w.M, "d": w.d, "V": w.V,
                        "K": 16, "r": w.r, "conv": [w.B, w.P, w.d], "parallelism": f"dp{world} (blocks)",
+                       "launch": "eager" if args.eager else f"cuda graphs of {chunk} cycles, PDL between kernels",
                        "l2": "inputs larger than L2 (W is %.0f MB > 126 MB)" % (2 * w.V * w.d / 1e6)},
             "e2e": {"value": aggregate(w.B, world, e_ms, e_steps), "unit": UNIT,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "path": "DraftCycle.run(): pinned H2D + conv + LM head + select/verify + D2H, host sync"},
             "gpu_launches": Step.LAUNCHES_PER_STEP * args.steps,
             "roofline": roof,
-            "stages_us": {"conv2tap": 1e3 * stage_ms[0], "lmhead_topk": 1e3 * stage_ms[1],
-                          "path_select": 1e3 * stage_ms[2], "verify": 1e3 * stage_ms[3],
-                          "select_plus_verify_share": (stage_ms[2] + stage_ms[3]) / (ms_max / args.steps)},
+            "stages_us": {**{n: 1e3 * t for n, t in zip(Step.STAGES, stage_ms)},
+                          "select_verify_share": stage_ms[2] / (ms_max / args.steps),
+                          "event_pair_overhead": 1e3 * ev_ms,
+                          "raw": {n: 1e3 * t for n, t in zip(Step.STAGES, raw_ms)},
+                          "samples": len(samples["lmhead_topk"]),
+                          "note": "durations net of the bracketing event-node pair (measured alone, 'raw' is gross)"},
             "clocks": clk.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -477,6 +540,7 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="launch each cycle eagerly instead of a CUDA graph")
     ap.add_argument("--ref-budget-s", type=float, default=120.0,
                     help="host seconds the --impl reference run aims to take")
     args = ap.parse_args(argv)

@@ -17,11 +17,14 @@ from ._binding import (  # noqa: F401
     dflash_lmhead_topk,
     dflash_lmhead_topk_workspace,
     dflash_path_select,
+    dflash_select_verify,
+    dflash_lmhead_topk_static,
     dflash_status_string,
     dflash_verify,
     lib,
     workspace,
 )
+from .cycle import DraftCycle  # noqa: F401,E402
 
 
 def bf16_tensor(bits: np.ndarray, device="cuda") -> torch.Tensor:

@@ -47,6 +47,8 @@ def _load():
         "dflash_lmhead_logits_debug": (i32, [vp, vp, i32, i32, i32, vp, vp, sz, vp, vp]),
         "dflash_path_select": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]),
         "dflash_verify": (i32, [vp, vp, i32, i32, vp, vp, vp]),
+        "dflash_select_verify": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]),
+        "dflash_lmhead_topk_static": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -178,6 +180,45 @@ def dflash_path_select(topk_logp, topk_idx, E, Msel, B, L, path_tok=None, path_s
         _ptr(path_slot), _ptr(path_score), _ptr(pair) if pair is not None and pair.numel() else None,
         _ptr(dev_status), _stream(stream)))
     return path_tok, path_slot, path_score, pair
+
+
+def dflash_select_verify(topk_logp, topk_idx, E, Msel, target, B, L, path_tok=None, path_slot=None,
+                         path_score=None, accept_len=None, next_token=None, dev_status=None, stream=None):
+    """Path selection and greedy verification of the chosen path in one kernel.
+    Returns (path_tok, path_slot, path_score, accept_len, next_token)."""
+    _need(topk_logp, "topk_logp", torch.float32, (B * L, K_TOP))
+    _need(topk_idx, "topk_idx", torch.int32, (B * L, K_TOP))
+    _need(E, "E", torch.bfloat16)
+    V, r = E.shape
+    _need(Msel, "Msel", torch.bfloat16, (r, r))
+    _need(target, "target", torch.int32, (B, L + 1))
+    dev = topk_logp.device
+    path_tok = _out(path_tok, "path_tok", torch.int32, (B, L), dev)
+    path_slot = _out(path_slot, "path_slot", torch.int32, (B, L), dev)
+    path_score = _out(path_score, "path_score", torch.float32, (B,), dev)
+    accept_len = _out(accept_len, "accept_len", torch.int32, (B,), dev)
+    next_token = _out(next_token, "next_token", torch.int32, (B,), dev)
+    _check("dflash_select_verify", lib.dflash_select_verify(
+        _ptr(topk_logp), _ptr(topk_idx), _ptr(E), _ptr(Msel), _ptr(target), B, L, K_TOP, r, V,
+        _ptr(path_tok), _ptr(path_slot), _ptr(path_score), _ptr(accept_len), _ptr(next_token),
+        _ptr(dev_status), _stream(stream)))
+    return path_tok, path_slot, path_score, accept_len, next_token
+
+
+def dflash_lmhead_topk_static(H, W, K=K_TOP, topk_logp=None, topk_idx=None, lse=None, dev_status=None,
+                              stream=None):
+    """dflash_lmhead_topk without a workspace (library-owned scratch; see the header)."""
+    _need(H, "H", torch.bfloat16)
+    _need(W, "W", torch.bfloat16)
+    M, d = H.shape
+    V = W.shape[0]
+    topk_logp = _out(topk_logp, "topk_logp", torch.float32, (M, K), H.device)
+    topk_idx = _out(topk_idx, "topk_idx", torch.int32, (M, K), H.device)
+    lse = _out(lse, "lse", torch.float32, (M,), H.device)
+    _check("dflash_lmhead_topk_static", lib.dflash_lmhead_topk_static(
+        _ptr(H), _ptr(W), M, V, d, K, _ptr(topk_logp), _ptr(topk_idx), _ptr(lse), _ptr(dev_status),
+        _stream(stream)))
+    return topk_logp, topk_idx, lse
 
 
 def dflash_verify(draft, target, accept_len=None, next_token=None, stream=None):

@@ -43,6 +43,8 @@ constexpr int UNROLL = 4;
 __global__ void __launch_bounds__(256) conv2tap_kernel(const uint4* __restrict__ x, const uint4* __restrict__ prev,
                                                        const uint4* __restrict__ a0, const uint4* __restrict__ a1,
                                                        uint4* __restrict__ y, int B, int P, int d8) {
+  pdl_wait();
+  pdl_trigger();
   const long long total = static_cast<long long>(B) * d8;
   for (long long id = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; id < total;
        id += static_cast<long long>(gridDim.x) * blockDim.x) {
@@ -106,8 +108,9 @@ extern "C" int dflash_conv2tap(const dflash_bf16* x, const dflash_bf16* prev, co
   long long blocks = (total + threads - 1) / threads;
   const long long cap = static_cast<long long>(sms) * 8;
   if (blocks > cap) blocks = cap;
-  dflash::conv::conv2tap_kernel<<<static_cast<int>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
-      reinterpret_cast<const uint4*>(x), reinterpret_cast<const uint4*>(prev), reinterpret_cast<const uint4*>(a0),
-      reinterpret_cast<const uint4*>(a1), reinterpret_cast<uint4*>(y), B, P, d8);
-  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
+  const cudaError_t e = dflash::launch_kernel(
+      dflash::conv::conv2tap_kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0,
+      static_cast<cudaStream_t>(stream), reinterpret_cast<const uint4*>(x), reinterpret_cast<const uint4*>(prev),
+      reinterpret_cast<const uint4*>(a0), reinterpret_cast<const uint4*>(a1), reinterpret_cast<uint4*>(y), B, P, d8);
+  return e == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }

@@ -182,6 +182,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Set-up above overlaps the previous kernel; global memory only from here.
+  pdl_wait();
   const uint64_t deadline = globaltimer_ns() + p.timeout_ns;
 
   int r0 = 0, r1 = 0;
@@ -432,6 +434,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   }
 
+  pdl_trigger();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -448,6 +451,8 @@ __global__ void __launch_bounds__(128) merge_kernel(const Partial* __restrict__ 
                                                     float* __restrict__ lse) {
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  pdl_wait();
+  pdl_trigger();
   if (row >= M) return;
   TopState st;
   st.reset();
@@ -657,21 +662,25 @@ static int launch(const dflash_bf16* H, const dflash_bf16* W, int M, int V, int 
                                          SMEM_BUDGET + 2048);
     });
     if (attr_err[0] != cudaSuccess) return DFLASH_ERR_CUDA;
-    lmhead_kernel<MODE_SWAP><<<pl.grid, NUM_THREADS, pl.smem, st>>>(ta, ta16, tb, p);
+    if (launch_kernel(lmhead_kernel<MODE_SWAP>, dim3(pl.grid), dim3(NUM_THREADS), pl.smem, st, ta, ta16, tb, p) !=
+        cudaSuccess)
+      return DFLASH_ERR_CUDA;
   } else {
     std::call_once(once[1], [] {
       attr_err[1] = cudaFuncSetAttribute(lmhead_kernel<MODE_LARGE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          SMEM_BUDGET + 2048);
     });
     if (attr_err[1] != cudaSuccess) return DFLASH_ERR_CUDA;
-    lmhead_kernel<MODE_LARGE><<<pl.grid, NUM_THREADS, pl.smem, st>>>(ta, ta16, tb, p);
+    if (launch_kernel(lmhead_kernel<MODE_LARGE>, dim3(pl.grid), dim3(NUM_THREADS), pl.smem, st, ta, ta16, tb, p) !=
+        cudaSuccess)
+      return DFLASH_ERR_CUDA;
   }
   if (cudaGetLastError() != cudaSuccess) return DFLASH_ERR_CUDA;
   if (z_dbg == nullptr) {
     const int rows_per_cta = 4;
-    merge_kernel<<<(M + rows_per_cta - 1) / rows_per_cta, 32 * rows_per_cta, 0, st>>>(p.part, M, p.P, topk_logp,
-                                                                                       topk_idx, lse);
-    if (cudaGetLastError() != cudaSuccess) return DFLASH_ERR_CUDA;
+    if (launch_kernel(merge_kernel, dim3((M + rows_per_cta - 1) / rows_per_cta), dim3(32 * rows_per_cta), 0, st,
+                      static_cast<const Partial*>(p.part), M, p.P, topk_logp, topk_idx, lse) != cudaSuccess)
+      return DFLASH_ERR_CUDA;
   }
   return DFLASH_OK;
 }

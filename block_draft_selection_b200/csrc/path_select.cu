@@ -9,21 +9,30 @@
 // Walk: delta_0 = 0, delta_{i+1}[k] = max_j delta_i[j] + S_i[j,k] (ties: lowest
 // j), end at argmax_k delta_{L-1}[k] (ties: lowest k), then backtrack.
 //
-// One CTA per block (1024 threads when there are few blocks, else 256):
-//   1. gather the 16*L candidate rows of E and the matrix M into shared memory
-//      (bf16, rows padded by 16 bytes so 16-byte loads of 8 neighbouring rows
-//      hit distinct banks);
-//   2. u_ij = e_{c_ij} M for all candidates of a chunk of positions (fp32),
-//      then the 16x16 pair scores of those positions, one (j,k) per thread;
-//   3. warp 0 walks the scores: lane (h,k) takes the max over j in half h of
-//      delta[j] + S[j,k], one xor-16 shuffle joins the halves, backpointers
-//      go to shared memory; then a 16-lane argmax and a backtrack.
+// One thread-block cluster of Q CTAs (256 threads each) per block; Q = 1 when
+// there are enough blocks to fill the GPU, else up to 8 so that a block's
+// pair scoring spreads over Q SMs:
+//   1. each CTA gathers the E rows of the positions it scores and the matrix
+//      M into shared memory (bf16, rows padded by 16 bytes so 16-byte loads
+//      of 8 neighbouring rows hit distinct banks);
+//   2. CTA q scores position pairs i = q, q+Q, ...: u_ij = e_{c_ij} M (fp32),
+//      then the 16x16 pair scores, one (j,k) per thread, written straight
+//      into the leader CTA's shared memory (distributed shared memory);
+//   3. after a cluster barrier, warp 0 of the leader walks the scores: lane
+//      (h,k) takes the max over j in half h of delta[j] + S[j,k], one xor-16
+//      shuffle joins the halves, backpointers go to shared memory; then a
+//      16-lane argmax, a backtrack and (optionally) greedy verification.
+#include <mutex>
+
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 
 namespace dflash {
 namespace sel {
 
-constexpr int MAX_THREADS = 1024;
+constexpr int THREADS = 256;
+constexpr int MAX_CLUSTER = 8;
 constexpr int KC = 16;
 constexpr int U_BUDGET = 48 * 1024;
 
@@ -67,10 +76,11 @@ __host__ __device__ inline Layout layout(int L, int r) {
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-__global__ void __launch_bounds__(MAX_THREADS) path_select_kernel(
+__global__ void __launch_bounds__(THREADS) path_select_kernel(
     const float* __restrict__ topk_logp, const int32_t* __restrict__ topk_idx, const uint16_t* __restrict__ E,
     const uint16_t* __restrict__ Msel, int L, int r, int V, int32_t* __restrict__ path_tok,
-    int32_t* __restrict__ path_slot, float* __restrict__ path_score, float* __restrict__ pair_dbg, int* status) {
+    int32_t* __restrict__ path_slot, float* __restrict__ path_score, float* __restrict__ pair_dbg, int* status,
+    const int32_t* __restrict__ target, int32_t* __restrict__ accept_len, int32_t* __restrict__ next_token, int Q) {
   extern __shared__ __align__(16) uint8_t smem[];
   const Layout lo = layout(L, r);
   uint16_t* Ms = reinterpret_cast<uint16_t*>(smem + lo.m_off);
@@ -81,16 +91,38 @@ __global__ void __launch_bounds__(MAX_THREADS) path_select_kernel(
   int* toks = reinterpret_cast<int*>(smem + lo.tok_off);
   int8_t* bps = reinterpret_cast<int8_t*>(smem + lo.bp_off);
 
-  const int b = blockIdx.x;
+  pdl_wait();
+  pdl_trigger();
+  const int b = blockIdx.x / Q;
+  const int q_rank = blockIdx.x - b * Q;  // rank in the cluster (clusters are Q consecutive CTAs)
   const int tid = threadIdx.x;
   const int nthr = blockDim.x;
   const int r8 = r / 8;
   const size_t row0 = static_cast<size_t>(b) * L;
+  const int npos = L - 1;
+  // Scores go to the leader's shared memory (this CTA's own when Q == 1).
+  // The leader's shared memory may be written only once every CTA of the
+  // cluster runs: arrive now, wait just before the first remote store.
+  float* S_out = Ss;
+  if (Q > 1) {
+    S_out = cooperative_groups::this_cluster().map_shared_rank(Ss, 0);
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+  }
+  // positions this CTA needs rows for: i and i+1 for every i = q_rank (mod Q)
+  auto needs_pos = [&](int i) {
+    if (Q == 1) return true;
+    const bool as_left = i < npos && (i % Q) == q_rank;
+    const bool as_right = i >= 1 && ((i - 1) % Q) == q_rank;
+    return as_left || as_right;
+  };
 
   // ---- 1. candidates, their E rows, and M into shared memory -------------
+  // One pass: every load here depends only on global inputs, so the index
+  // reads, the E-row gathers that follow them and the copy of M are all in
+  // flight together.
   for (int q = tid; q < L * KC; q += nthr) {
-    lps[q] = topk_logp[row0 * KC + q];
-    int c = topk_idx[row0 * KC + q];
+    lps[q] = __ldg(topk_logp + row0 * KC + q);
+    int c = __ldg(topk_idx + row0 * KC + q);
     if (c < 0 || c >= V) {
       set_status(status, DFLASH_ERR_BAD_INDEX);
       c = 0;
@@ -102,27 +134,34 @@ __global__ void __launch_bounds__(MAX_THREADS) path_select_kernel(
     uint4* Mv = reinterpret_cast<uint4*>(Ms);
     for (int q = tid; q < r * r8; q += nthr) Mv[q] = __ldg(Mg + q);
   }
-  __syncthreads();
   for (int q = tid; q < L * KC * r8; q += nthr) {
     const int cand = q / r8;
     const int v8 = q - cand * r8;
-    const uint4 val = __ldg(reinterpret_cast<const uint4*>(E + static_cast<size_t>(toks[cand]) * r) + v8);
+    if (!needs_pos(cand / KC)) continue;
+    int c = __ldg(topk_idx + row0 * KC + cand);
+    c = (c < 0 || c >= V) ? 0 : c;
+    const uint4 val = __ldg(reinterpret_cast<const uint4*>(E + static_cast<size_t>(c) * r) + v8);
     *reinterpret_cast<uint4*>(Es + static_cast<size_t>(cand) * lo.rp + v8 * 8) = val;
   }
   __syncthreads();
 
-  // ---- 2. pair scores, a chunk of positions at a time --------------------
-  const int npos = L - 1;
-  for (int i0 = 0; i0 < npos; i0 += lo.pc) {
-    const int pcn = min(lo.pc, npos - i0);
+  if (Q > 1) asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+
+  // ---- 2. pair scores, a chunk of this CTA's positions at a time ----------
+  // This CTA's positions are i = q_rank + Q*m; chunk index ii counts m.
+  const int my_npos = npos > q_rank ? (npos - q_rank + Q - 1) / Q : 0;
+  for (int m0 = 0; m0 < my_npos; m0 += lo.pc) {
+    const int pcn = min(lo.pc, my_npos - m0);
     // u[ii][j][t] = sum_s e_{c_(i0+ii),j}[s] * M[s][t], 8 outputs per item
     for (int q = tid; q < pcn * KC * r8; q += nthr) {
       const int tg = q % r8;
       const int jj = q / r8;  // (ii * 16 + j)
       const int ii = jj / KC;
       const int j = jj - ii * KC;
-      const uint16_t* er = Es + static_cast<size_t>((i0 + ii) * KC + j) * lo.rp;
+      const int i = q_rank + Q * (m0 + ii);
+      const uint16_t* er = Es + static_cast<size_t>(i * KC + j) * lo.rp;
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
       for (int s = 0; s < r; ++s) {
         const float es = __uint_as_float(static_cast<uint32_t>(er[s]) << 16);
         const uint4 mv = *reinterpret_cast<const uint4*>(Ms + static_cast<size_t>(s) * r + tg * 8);
@@ -144,10 +183,11 @@ __global__ void __launch_bounds__(MAX_THREADS) path_select_kernel(
       const int k = q % KC;
       const int j = (q / KC) % KC;
       const int ii = q / (KC * KC);
-      const int i = i0 + ii;
+      const int i = q_rank + Q * (m0 + ii);
       const float* ur = Us + static_cast<size_t>(ii * KC + j) * lo.up;
       const uint16_t* er = Es + static_cast<size_t>((i + 1) * KC + k) * lo.rp;
       float acc = 0.f;
+#pragma unroll 4
       for (int t = 0; t < r; t += 8) {
         const float4 u0 = *reinterpret_cast<const float4*>(ur + t);
         const float4 u1 = *reinterpret_cast<const float4*>(ur + t + 4);
@@ -162,13 +202,17 @@ __global__ void __launch_bounds__(MAX_THREADS) path_select_kernel(
         acc = fmaf(u1.w, bf_hi(ev.w), acc);
       }
       const float sc = (lps[i * KC + j] + lps[(i + 1) * KC + k]) + acc;
-      Ss[(i * KC + j) * KC + k] = sc;
+      S_out[(i * KC + j) * KC + k] = sc;
       if (pair_dbg) pair_dbg[((static_cast<size_t>(b) * npos + i) * KC + j) * KC + k] = sc;
     }
     __syncthreads();
   }
 
-  // ---- 3. max-sum walk (warp 0) -------------------------------------------
+  // ---- 3. max-sum walk (warp 0 of the leader) -----------------------------
+  if (Q > 1) {
+    cooperative_groups::this_cluster().sync();  // every CTA's scores have landed
+    if (q_rank != 0) return;
+  }
   if (tid < 32) {
     const int lane = tid;
     const int k = lane & 15;
@@ -211,17 +255,75 @@ __global__ void __launch_bounds__(MAX_THREADS) path_select_kernel(
         bk = k2;
       }
     }
+    // Backtrack (lane 0) into shared memory, then lane i writes position i.
+    int* pslot = reinterpret_cast<int*>(Us);  // u is no longer needed
     if (lane == 0) {
       int slot = npos > 0 ? bk : 0;
-      const float score = npos > 0 ? bv : 0.f;
       for (int i = L - 1; i >= 0; --i) {
-        path_tok[row0 + i] = toks[i * KC + slot];
-        if (path_slot) path_slot[row0 + i] = slot;
+        pslot[i] = slot;
         if (i > 0) slot = bps[(i - 1) * KC + slot];
       }
-      if (path_score) path_score[b] = score;
+      if (path_score) path_score[b] = npos > 0 ? bv : 0.f;
+    }
+    __syncwarp();
+    const bool in_block = lane < L;
+    const int my_slot = in_block ? pslot[lane] : 0;
+    const int my_tok = in_block ? toks[lane * KC + my_slot] : 0;
+    if (in_block) {
+      path_tok[row0 + lane] = my_tok;
+      if (path_slot) path_slot[row0 + lane] = my_slot;
+    }
+    // ---- 4. optional greedy verification of the selected path ------------
+    if (target != nullptr) {
+      const int32_t* tg = target + static_cast<size_t>(b) * (L + 1);
+      const bool differs = in_block && my_tok != __ldg(tg + lane);
+      const unsigned mask = __ballot_sync(0xffffffffu, differs);
+      const int n = mask ? __ffs(mask) - 1 : L;
+      if (lane == 0) {
+        accept_len[b] = n + 1;
+        next_token[b] = __ldg(tg + n);
+      }
     }
   }
+}
+
+}  // namespace sel
+}  // namespace dflash
+
+namespace dflash {
+namespace sel {
+
+static int launch(const float* topk_logp, const int32_t* topk_idx, const dflash_bf16* E, const dflash_bf16* Msel,
+                  int B, int L, int K, int r, int V, int32_t* path_tok, int32_t* path_slot, float* path_score,
+                  float* pair_scores_dbg, const int32_t* target, int32_t* accept_len, int32_t* next_token,
+                  int* dev_status, void* stream) {
+  if (!topk_logp || !topk_idx || !E || !Msel || !path_tok) return DFLASH_ERR_INVALID_ARG;
+  if (K != KC || B < 1 || L < 1 || L > 16 || r < 8 || r > 128 || r % 8 != 0 || V < 1)
+    return DFLASH_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(E) | reinterpret_cast<uintptr_t>(Msel)) & 15) return DFLASH_ERR_INVALID_ARG;
+  const Layout lo = layout(L, r);
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(path_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  });
+  if (attr_err != cudaSuccess) return DFLASH_ERR_CUDA;
+  // Few blocks: one cluster of up to 8 CTAs per block spreads its pair scoring
+  // over several SMs (latency); many blocks fill the GPU one CTA per block.
+  int sms = 148, dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int Q = 1;
+  if (B * 2 < sms && L > 2) {
+    Q = L - 1 < MAX_CLUSTER ? L - 1 : MAX_CLUSTER;
+    while (Q > 1 && static_cast<long long>(B) * Q > sms) --Q;
+  }
+  const cudaError_t e =
+      launch_kernel_cluster(path_select_kernel, dim3(B * Q), dim3(THREADS), lo.total, static_cast<cudaStream_t>(stream),
+                            Q, topk_logp, topk_idx, reinterpret_cast<const uint16_t*>(E),
+                            reinterpret_cast<const uint16_t*>(Msel), L, r, V, path_tok, path_slot, path_score,
+                            pair_scores_dbg, dev_status, target, accept_len, next_token, Q);
+  return e == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }
 
 }  // namespace sel
@@ -231,23 +333,15 @@ extern "C" int dflash_path_select(const float* topk_logp, const int32_t* topk_id
                                   const dflash_bf16* Msel, int B, int L, int K, int r, int V, int32_t* path_tok,
                                   int32_t* path_slot, float* path_score, float* pair_scores_dbg, int* dev_status,
                                   void* stream) {
-  using namespace dflash::sel;
-  if (!topk_logp || !topk_idx || !E || !Msel || !path_tok) return DFLASH_ERR_INVALID_ARG;
-  if (K != KC || B < 1 || L < 1 || L > 16 || r < 8 || r > 128 || r % 8 != 0 || V < 1)
-    return DFLASH_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(E) | reinterpret_cast<uintptr_t>(Msel)) & 15) return DFLASH_ERR_INVALID_ARG;
-  const Layout lo = layout(L, r);
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(path_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) !=
-        cudaSuccess)
-      return DFLASH_ERR_CUDA;
-    attr_done = true;
-  }
-  // Few blocks: spread each block's candidate work over more threads (latency);
-  // many blocks: 256 threads so several CTAs share an SM.
-  const int threads = B < 128 ? 1024 : 256;
-  path_select_kernel<<<B, threads, lo.total, static_cast<cudaStream_t>(stream)>>>(
-      topk_logp, topk_idx, E, Msel, L, r, V, path_tok, path_slot, path_score, pair_scores_dbg, dev_status);
-  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
+  return dflash::sel::launch(topk_logp, topk_idx, E, Msel, B, L, K, r, V, path_tok, path_slot, path_score,
+                             pair_scores_dbg, nullptr, nullptr, nullptr, dev_status, stream);
+}
+
+extern "C" int dflash_select_verify(const float* topk_logp, const int32_t* topk_idx, const dflash_bf16* E,
+                                    const dflash_bf16* Msel, const int32_t* target, int B, int L, int K, int r,
+                                    int V, int32_t* path_tok, int32_t* path_slot, float* path_score,
+                                    int32_t* accept_len, int32_t* next_token, int* dev_status, void* stream) {
+  if (!target || !accept_len || !next_token) return DFLASH_ERR_INVALID_ARG;
+  return dflash::sel::launch(topk_logp, topk_idx, E, Msel, B, L, K, r, V, path_tok, path_slot, path_score,
+                             nullptr, target, accept_len, next_token, dev_status, stream);
 }

@@ -16,6 +16,8 @@ __global__ void __launch_bounds__(32 * WARPS) verify_kernel(const int32_t* __res
                                                              const int32_t* __restrict__ target, int B, int L,
                                                              int32_t* __restrict__ accept_len,
                                                              int32_t* __restrict__ next_token) {
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.x * WARPS + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (b >= B) return;
@@ -36,7 +38,8 @@ extern "C" int dflash_verify(const int32_t* draft, const int32_t* target, int B,
                              int32_t* next_token, void* stream) {
   using namespace dflash::ver;
   if (!draft || !target || !accept_len || !next_token || B < 1 || L < 1 || L > 32) return DFLASH_ERR_INVALID_ARG;
-  verify_kernel<<<(B + WARPS - 1) / WARPS, 32 * WARPS, 0, static_cast<cudaStream_t>(stream)>>>(
-      draft, target, B, L, accept_len, next_token);
-  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
+  const cudaError_t e = dflash::launch_kernel(verify_kernel, dim3((B + WARPS - 1) / WARPS), dim3(32 * WARPS), 0,
+                                              static_cast<cudaStream_t>(stream), draft, target, B, L, accept_len,
+                                              next_token);
+  return e == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }

@@ -160,6 +160,19 @@ int dflash_path_select(const float* topk_logp, const int32_t* topk_idx, const df
                        float* pair_scores_dbg, int* dev_status, void* stream);
 
 /*
+ * dflash_path_select followed by greedy verification of the selected path,
+ * in one kernel ("DFlash 2: Keep Drafting Parallel", section "a lightweight
+ * path selector" and Table 1's caption): the same outputs as
+ * dflash_path_select (without the pair-score dump) plus, for the chosen
+ * path, accept_len [B] and next_token [B] exactly as dflash_verify defines
+ * them against target [B, L+1] int32.  1 <= L <= 16.
+ */
+int dflash_select_verify(const float* topk_logp, const int32_t* topk_idx, const dflash_bf16* E,
+                         const dflash_bf16* Msel, const int32_t* target, int B, int L, int K, int r, int V,
+                         int32_t* path_tok, int32_t* path_slot, float* path_score, int32_t* accept_len,
+                         int32_t* next_token, int* dev_status, void* stream);
+
+/*
  * Greedy verification.
  * "DFlash 2: Keep Drafting Parallel", Table 1 caption: the accepted length
  * includes the verifier's next token.  With n the first i where

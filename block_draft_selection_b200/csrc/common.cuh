@@ -183,6 +183,12 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   return p;
 }
 
+__device__ __forceinline__ uint64_t l2_policy_evict_normal() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
@@ -285,6 +291,79 @@ __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
 
 __device__ __forceinline__ int elect_lane0() { return (threadIdx.x & 31) == 0; }
 
+// ------------------------------------------------- 2-CTA (cta_group::2) ----
+// A cluster of two CTAs shares one tcgen05.mma of M = 256: each CTA stages
+// half of A (128 rows) and half of B (N/2 rows) in its own shared memory at
+// the same offsets; the leader (rank 0) issues the MMA and each CTA's TMEM
+// receives its 128 rows of D.
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// shared::cluster address of the same shared-memory offset in CTA `rank`.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Arrive on an mbarrier of another CTA of the cluster.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// TMA load into this CTA's shared memory whose byte count completes on the
+// leader's barrier (`bar_cluster` is a shared::cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster, int c0,
+                                                 int c1, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive once on the barrier at this offset in every CTA of `cta_mask` when
+// the pair MMAs issued so far by this thread have completed.
+__device__ __forceinline__ void umma_commit_pair_multicast(uint32_t bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(cta_mask)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
 // ------------------------------------------------------ top-16 in registers --
 
 constexpr int KTOP = 16;
@@ -321,6 +400,30 @@ struct TopState {
     bool ahead[KTOP];
 #pragma unroll
     for (int k = 0; k < KTOP; ++k) ahead[k] = better(v[k], i[k], x, ix);
+    float nv[KTOP];
+    int ni[KTOP];
+    nv[0] = ahead[0] ? v[0] : x;
+    ni[0] = ahead[0] ? i[0] : ix;
+#pragma unroll
+    for (int k = 1; k < KTOP; ++k) {
+      nv[k] = ahead[k] ? v[k] : (ahead[k - 1] ? x : v[k - 1]);
+      ni[k] = ahead[k] ? i[k] : (ahead[k - 1] ? ix : i[k - 1]);
+    }
+#pragma unroll
+    for (int k = 0; k < KTOP; ++k) {
+      v[k] = nv[k];
+      i[k] = ni[k];
+    }
+  }
+
+  // Insert for a scan that visits indices in increasing order: any entry
+  // already in the list has a smaller index than `ix`, so an equal value stays
+  // ahead and every order test is a single value compare.
+  __device__ __forceinline__ void insert_scan(float x, int ix) {
+    if (!(x > v[KTOP - 1])) return;
+    bool ahead[KTOP];
+#pragma unroll
+    for (int k = 0; k < KTOP; ++k) ahead[k] = v[k] >= x;
     float nv[KTOP];
     int ni[KTOP];
     nv[0] = ahead[0] ? v[0] : x;

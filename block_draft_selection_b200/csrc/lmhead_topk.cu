@@ -8,28 +8,33 @@
 //   top-16 of z[m,:] (value desc, index asc), logp = z - lse.
 //
 // Kernel 1 (lmhead_kernel) is a persistent, warp-specialised tcgen05 GEMM:
-//   warp 0      TMA producer: 128-byte-swizzled K-major tiles of W and H into
+//   warp 0      TMA producer: 128-byte-swizzled K-major tiles of H and W into
 //               a ring of shared-memory stages (mbarrier transaction counts)
 //   warp 1      MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16 -> fp32) into
 //               a double-buffered TMEM accumulator; owns the TMEM allocation
-//   warps 2..5  epilogue: tcgen05.ld the accumulator, keep an online
-//               (max, sum exp) and a register-resident sorted top-16 per row,
-//               write one partial record per (row, slot)
-// Two tile orientations:
-//   SWAP  (M <= 128, weight streaming): the MMA's M side is 128 vocabulary
-//         rows of W, its N side the M tokens padded to 16.  Each CTA owns one
-//         contiguous, balanced vocabulary range (16-row granularity; a ragged
-//         last tile is fetched as 16-row boxes so no byte of W is read twice).
-//         The epilogue transposes the tile through shared memory so threads
-//         own tokens.  One partial per (row, CTA).
-//   LARGE (M > 128, tensor bound): the MMA's M side is 128 token rows, its N
-//         side 256 vocabulary columns; TMEM lane = token row, so each thread
-//         scans its row directly.  Tiles are visited vocabulary-major so the
-//         CTAs working at one time share W tiles through L2.  One partial per
-//         (row, vocabulary tile).
+//   warps 2..9  epilogue: TMEM lane = token row; two warps share each lane
+//               quarter and split the tile's vocabulary columns; each thread
+//               keeps an online (max, sum exp) and a register-resident sorted
+//               top-16 and writes one partial record per (row, slot, half)
+// The MMA's M side is always token rows and its N side up to 256 vocabulary
+// rows of W: a tcgen05.mma of M = 128 costs about the same time for any N up
+// to 256, so W goes on the N side where each instruction consumes 256 rows.
+//   STREAM (M <= 128, weight streaming): one token tile (the A box holds the
+//          M rows rounded up to 16; the MMA's other rows are never read back).
+//          Each CTA owns one contiguous, balanced vocabulary range at 16-row
+//          granularity; a ragged last tile is fetched as 16-row boxes and
+//          multiplied with a narrower N, so no byte of W is read twice.
+//   LARGE  (M > 128, tensor bound): token tiles of 128 rows, or 256 rows on a
+//          cluster of two CTAs sharing one tcgen05.mma.cta_group::2 ("pair":
+//          each CTA stages half of A and half of B, the leader issues the MMA
+//          and each CTA's TMEM receives its 128 rows of D).  Tiles are either
+//          vocabulary-strided (W shared through L2 across concurrent token
+//          tiles) or long runs of one token tile over a vocabulary range.
+// No load uses cluster multicast: every CTA fetches its own tiles.
 // Kernel 2 (merge_kernel) folds a row's partials: one warp per row.
 #include <cstdio>
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -39,42 +44,47 @@ namespace lm {
 
 constexpr int BK = 64;                  // bf16 per K stage = one 128-byte swizzle row
 constexpr int UMMA_K = 16;              // K per tcgen05.mma kind::f16
-constexpr int A_ROWS = 128;             // MMA M
-constexpr int A_STAGE_BYTES = A_ROWS * BK * 2;
-constexpr int LARGE_N = 256;            // MMA N in LARGE mode
-constexpr int NUM_THREADS = 192;
-constexpr int EPI_THREADS = 128;
+constexpr int A_ROWS = 128;             // token rows per CTA and MMA M of one CTA
+constexpr int TILE_N = 256;             // vocabulary rows per tile (MMA N)
+constexpr int EPI_WARPS = 8;
+constexpr int EPI_THREADS = 32 * EPI_WARPS;
+constexpr int NUM_THREADS = 64 + EPI_THREADS;
 constexpr int SMEM_BUDGET = 224 * 1024;
+constexpr int MMA_A_SPAN = A_ROWS * BK * 2;  // shared bytes one MMA reads from an A stage
 
-enum { MODE_SWAP = 0, MODE_LARGE = 1 };
-// LARGE-orientation tile schedules:
-//  STRIDED  tile t = cta + k * grid in vocabulary-major order: the CTAs running
+enum { MODE_STREAM = 0, MODE_LARGE = 1 };
+// LARGE-orientation tile schedules (over work units = CTAs, or CTA pairs):
+//  BLOCKS   the (token tile, block of R consecutive vocabulary tiles) jobs,
+//           ordered block-major, go to units round-robin: the units running
 //           at one time cover a narrow vocabulary window (W tiles are shared
-//           through L2); each tile starts a fresh candidate list.
-//  RUNS     CTA c owns m-tile (c % m_tiles) over one contiguous vocabulary range
-//           (range c / m_tiles of nr); the CTAs owning one range walk it in
-//           lockstep (W shared through L2) and each keeps its candidate list
-//           across the whole range, so few values reach the insertion code.
-enum { SCHED_STRIDED = 0, SCHED_RUNS = 1 };
+//           through L2 by the token tiles) and each job keeps one candidate
+//           list over its R tiles.  R = 1 is a plain vocabulary-strided walk.
+//  RUNS     unit u owns token tile (u % m_tiles) over one contiguous
+//           vocabulary range (range u / m_tiles of nr); the units owning one
+//           range walk it in lockstep (W shared through L2) and each keeps
+//           its candidate list across the whole range.
+// The host picks the schedule with the fewest tiles on the busiest unit,
+// charging short runs a little for their candidate-list restarts.
+enum { SCHED_BLOCKS = 0, SCHED_RUNS = 1 };
 
 struct Params {
   int M, V, d;
   int num_kc;        // K stages per tile = ceil(d / 64)
   int stages;        // shared-memory ring depth
-  int n_mma;         // MMA N
-  int tmem_cols;     // allocated TMEM columns (power of two >= 32)
-  int buf_cols;      // TMEM columns per accumulator buffer
-  int b_stage_bytes; // shared bytes of one B stage
-  int b_tx_bytes;    // TMA bytes landing in one B stage
-  // SWAP
-  int units;         // ceil(V / 16)
-  int g;             // epilogue threads per token
-  int t_stride;      // floats per token row of the transpose buffer
-  int t_bytes;
+  int a_box;         // A rows this CTA loads per stage (STREAM: M rounded up to 16)
+  int a_stage_bytes;
+  int b_rows;        // B rows this CTA loads per full tile (its half in a pair)
+  int b_stage_bytes;
+  int tmem_cols;
+  // STREAM
+  int units;         // 16-row vocabulary units
   // LARGE
-  int m_tiles, v_tiles;
-  int sched;         // SCHED_STRIDED or SCHED_RUNS
-  int nr;            // SCHED_RUNS: vocabulary ranges per m-tile
+  int m_tiles, v_tiles;  // token tiles of 128 rows (256 for pairs), vocabulary tiles of 256
+  int sched;
+  int nr;            // RUNS: vocabulary ranges per token tile
+  int R;             // BLOCKS: vocabulary tiles per job
+  int n_vblocks;     // BLOCKS: ceil(v_tiles / R)
+  int b_widths[4];   // STREAM: the tile widths, one tensor map each
   // outputs
   Partial* part;     // [M][P]
   int P;
@@ -84,15 +94,18 @@ struct Params {
 };
 
 struct SmemLayout {
-  uint32_t a, b, t, bars, misc, total;
+  uint32_t a, b, bars, misc, total;
 };
 
 __host__ __device__ inline SmemLayout smem_layout(const Params& p) {
   SmemLayout s;
   s.a = 0;
-  s.b = s.a + p.stages * A_STAGE_BYTES;
-  s.t = s.b + p.stages * p.b_stage_bytes;
-  s.bars = s.t + p.t_bytes;
+  s.b = s.a + p.stages * p.a_stage_bytes;
+  // an MMA reads a full 128-row span from its A stage: keep that span inside
+  // the allocation (rows beyond the loaded box are never read back)
+  uint32_t b_min = (p.stages - 1) * p.a_stage_bytes + MMA_A_SPAN;
+  if (s.b < b_min) s.b = (b_min + 1023) & ~1023u;
+  s.bars = s.b + p.stages * p.b_stage_bytes;
   s.misc = s.bars + (2 * p.stages + 5) * 8;
   s.total = s.misc + 16;
   return s;
@@ -100,46 +113,91 @@ __host__ __device__ inline SmemLayout smem_layout(const Params& p) {
 
 // ------------------------------------------------------------ tile walks ---
 
-// SWAP: this CTA's balanced vocabulary range [r0, r1), a multiple of 16 rows.
-__device__ __forceinline__ void swap_range(const Params& p, int& r0, int& r1) {
-  const long long G = gridDim.x;
-  const long long c = blockIdx.x;
-  r0 = static_cast<int>((c * p.units) / G) * 16;
-  r1 = static_cast<int>(((c + 1) * p.units) / G) * 16;
-}
+template <bool PAIR>
+__device__ __forceinline__ int unit_id() { return PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x); }
+template <bool PAIR>
+__device__ __forceinline__ int unit_count() { return PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x); }
 
-// LARGE: the k-th tile of this CTA; false past the end.  `slot` names the
-// partial record the tile's run writes; first/last mark the run's ends.
-__device__ __forceinline__ bool large_tile(const Params& p, int k, int& mt, int& vt, int& slot, bool& first,
-                                           bool& last) {
+struct Tile {
+  int a_row;   // first token row of this CTA's A rows (and of its TMEM lanes)
+  int b_row;   // first W row this CTA loads
+  int n_cols;  // MMA N (vocabulary rows of the tile)
+  int v0;      // vocabulary index of accumulator column 0
+  int slot;    // partial-record slot of the tile's run
+  bool first, last;
+};
+
+// The k-th tile of this CTA; false past the end.
+template <int MODE, bool PAIR>
+__device__ __forceinline__ bool get_tile(const Params& p, int k, uint32_t rank, Tile& t) {
+  if (MODE == MODE_STREAM) {
+    // The range is cut into the fewest tiles of at most 256 rows, all of
+    // (nearly) equal width: every tile costs a full K loop of MMAs whatever
+    // its width, so no CTA carries a sliver tile.
+    const long long G = gridDim.x, c = blockIdx.x;
+    const int u0 = static_cast<int>((c * p.units) / G);
+    const int u1 = static_cast<int>(((c + 1) * p.units) / G);
+    const int nt = (u1 - u0 + TILE_N / 16 - 1) / (TILE_N / 16);
+    const int wu = nt > 0 ? (u1 - u0 + nt - 1) / nt : 0;  // units per tile
+    const int t0 = (u0 + k * wu) * 16;
+    if (k >= nt || t0 >= u1 * 16) return false;
+    t.a_row = 0;
+    t.b_row = t0;
+    t.n_cols = min(wu * 16, u1 * 16 - t0);
+    t.v0 = t0;
+    t.slot = blockIdx.x;
+    t.first = k == 0;
+    t.last = k == nt - 1 || t0 + wu * 16 >= u1 * 16;
+    return true;
+  }
+  const int u = unit_id<PAIR>();
+  int mt, vt;
   if (p.sched == SCHED_RUNS) {
-    const int c = blockIdx.x;
-    mt = c % p.m_tiles;
-    const int r = c / p.m_tiles;
+    mt = u % p.m_tiles;
+    const int r = u / p.m_tiles;
     const int lo = static_cast<int>(static_cast<long long>(r) * p.v_tiles / p.nr);
     const int hi = static_cast<int>(static_cast<long long>(r + 1) * p.v_tiles / p.nr);
     vt = lo + k;
     if (vt >= hi) return false;
-    slot = r;
-    first = k == 0;
-    last = vt == hi - 1;
-    return true;
+    t.slot = r;
+    t.first = k == 0;
+    t.last = vt == hi - 1;
+  } else {
+    // k-th tile of this unit: job j = u + (k / R') * units ... walked job by
+    // job; each job covers R tiles (the last vocabulary block may be shorter)
+    const long long jobs = static_cast<long long>(p.m_tiles) * p.n_vblocks;
+    long long job = u;
+    int kk = k;
+    for (;;) {
+      if (job >= jobs) return false;
+      const int vb = static_cast<int>(job / p.m_tiles);
+      const int len = min(p.R, p.v_tiles - vb * p.R);
+      if (kk < len) {
+        mt = static_cast<int>(job - static_cast<long long>(vb) * p.m_tiles);
+        vt = vb * p.R + kk;
+        t.slot = vb;
+        t.first = kk == 0;
+        t.last = kk == len - 1;
+        break;
+      }
+      kk -= len;
+      job += unit_count<PAIR>();
+    }
   }
-  const long long t = blockIdx.x + static_cast<long long>(k) * gridDim.x;
-  if (t >= static_cast<long long>(p.m_tiles) * p.v_tiles) return false;
-  vt = static_cast<int>(t / p.m_tiles);
-  mt = static_cast<int>(t - static_cast<long long>(vt) * p.m_tiles);
-  slot = vt;
-  first = last = true;
+  t.a_row = mt * (PAIR ? 2 * A_ROWS : A_ROWS) + static_cast<int>(rank) * A_ROWS;
+  t.b_row = vt * TILE_N + static_cast<int>(rank) * p.b_rows;
+  t.n_cols = TILE_N;
+  t.v0 = vt * TILE_N;
   return true;
 }
 
 // ------------------------------------------------------------ kernel -------
 
-template <int MODE>
+template <int MODE, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    lmhead_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a16,
-                  const __grid_constant__ CUtensorMap tm_b, const Params p) {
+    lmhead_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                  const __grid_constant__ CUtensorMap tm_w1, const __grid_constant__ CUtensorMap tm_w2,
+                  const __grid_constant__ CUtensorMap tm_w3, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -153,10 +211,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t drain_bar = bar0 + 8u * (2 * p.stages + 4);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 4);
-  volatile int* epi_ok = reinterpret_cast<volatile int*>(smem + L.misc + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
@@ -165,318 +224,264 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), EPI_THREADS);
+      mbar_init(tempty_bar(b), PAIR ? 2 * EPI_THREADS : EPI_THREADS);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
-    *epi_ok = 1;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tm_a);
-    prefetch_tmap(&tm_a16);
     prefetch_tmap(&tm_b);
+    if (MODE == MODE_STREAM) {
+      prefetch_tmap(&tm_w1);
+      prefetch_tmap(&tm_w2);
+      prefetch_tmap(&tm_w3);
+    }
   }
-  if (warp == 1) tmem_alloc(smem_addr(tmem_slot), p.tmem_cols);
+  if (warp == 1) {
+    if (PAIR)
+      tmem_alloc_pair(smem_addr(tmem_slot), p.tmem_cols);
+    else
+      tmem_alloc(smem_addr(tmem_slot), p.tmem_cols);
+  }
   tc_fence_before();
   __syncthreads();
+  __syncwarp();
+  if (PAIR) cluster_sync_all();  // both CTAs' barriers exist before any remote signal
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // Set-up above overlaps the previous kernel; global memory only from here.
   pdl_wait();
   const uint64_t deadline = globaltimer_ns() + p.timeout_ns;
 
-  int r0 = 0, r1 = 0;
-  if (MODE == MODE_SWAP) swap_range(p, r0, r1);
-
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
       const uint64_t pol_stream = l2_policy_evict_first();
       const uint64_t pol_keep = l2_policy_evict_last();
+      const uint64_t pol_normal = l2_policy_evict_normal();
+      // W is read once when streaming; shared by concurrent token tiles otherwise
+      const uint64_t pol_w = MODE == MODE_STREAM ? pol_stream : pol_normal;
       int s = 0;
       uint32_t ph = 0;
       uint32_t issued_mask = 0, issued_par = 0;
       bool ok = true;
-      if (MODE == MODE_SWAP) {
-        for (int t0 = r0; ok && t0 < r1; t0 += A_ROWS) {
-          const int rows = min(A_ROWS, r1 - t0);
-          for (int kc = 0; kc < p.num_kc; ++kc) {
-            if (!mbar_wait(empty_bar(s), ph ^ 1u, deadline, abort_flag, p.status)) {
-              ok = false;
-              break;
-            }
-            const uint32_t fb = full_bar(s);
-            mbar_arrive_expect_tx(fb, static_cast<uint32_t>(rows * BK * 2 + p.b_tx_bytes));
-            const uint32_t a_dst = sbase + L.a + s * A_STAGE_BYTES;
-            if (rows == A_ROWS) {
-              tma_load_2d_hint(a_dst, &tm_a, fb, kc * BK, t0, pol_stream);
-            } else {
-              for (int j = 0; j < rows / 16; ++j)
-                tma_load_2d_hint(a_dst + j * 16 * BK * 2, &tm_a16, fb, kc * BK, t0 + 16 * j, pol_stream);
-            }
-            tma_load_2d_hint(sbase + L.b + s * p.b_stage_bytes, &tm_b, fb, kc * BK, 0, pol_keep);
-            issued_mask |= 1u << s;
-            issued_par = (issued_par & ~(1u << s)) | (ph << s);
-            if (++s == p.stages) { s = 0; ph ^= 1u; }
+      auto load = [&](uint32_t dst, const CUtensorMap* m, uint32_t fb, int c0, int c1, uint64_t pol) {
+        if (PAIR)
+          tma_load_2d_pair(dst, m, mapa_shared(fb, 0), c0, c1, pol);
+        else
+          tma_load_2d_hint(dst, m, fb, c0, c1, pol);
+      };
+      Tile t;
+      for (int k = 0; ok && get_tile<MODE, PAIR>(p, k, rank, t); ++k) {
+        // bytes landing on the leader's barrier per stage (both CTAs of a pair)
+        const int b_rows_here = MODE == MODE_STREAM ? t.n_cols : p.b_rows;
+        const uint32_t tx = static_cast<uint32_t>((PAIR ? 2 : 1) * (p.a_box + b_rows_here) * BK * 2);
+        for (int kc = 0; kc < p.num_kc; ++kc) {
+          if (!mbar_wait(empty_bar(s), ph ^ 1u, deadline, abort_flag, p.status)) {
+            ok = false;
+            break;
           }
-        }
-      } else {
-        int mt, vt, slot;
-        bool first, last;
-        for (int k = 0; ok && large_tile(p, k, mt, vt, slot, first, last); ++k) {
-          for (int kc = 0; kc < p.num_kc; ++kc) {
-            if (!mbar_wait(empty_bar(s), ph ^ 1u, deadline, abort_flag, p.status)) {
-              ok = false;
-              break;
-            }
-            const uint32_t fb = full_bar(s);
-            mbar_arrive_expect_tx(fb, static_cast<uint32_t>(A_STAGE_BYTES + p.b_tx_bytes));
-            tma_load_2d_hint(sbase + L.a + s * A_STAGE_BYTES, &tm_a, fb, kc * BK, mt * A_ROWS, pol_keep);
-            // W tiles are shared by the m-tiles running at the same time: default L2 policy.
-            tma_load_2d(sbase + L.b + s * p.b_stage_bytes, &tm_b, fb, kc * BK, vt * LARGE_N);
-            issued_mask |= 1u << s;
-            issued_par = (issued_par & ~(1u << s)) | (ph << s);
-            if (++s == p.stages) { s = 0; ph ^= 1u; }
+          const uint32_t fb = full_bar(s);
+          if (leader) mbar_arrive_expect_tx(fb, tx);
+          load(sbase + L.a + s * p.a_stage_bytes, &tm_a, fb, kc * BK, t.a_row, pol_keep);
+          const uint32_t b_dst = sbase + L.b + s * p.b_stage_bytes;
+          // one box per stage: the map whose box height is this tile's width
+          // (STREAM tiles take one of at most four widths, known on the host)
+          const CUtensorMap* mb = &tm_b;   // LARGE: the full tile; STREAM: width b_widths[0]
+          if (MODE == MODE_STREAM) {
+            if (b_rows_here == p.b_widths[1]) mb = &tm_w1;
+            else if (b_rows_here == p.b_widths[2]) mb = &tm_w2;
+            else if (b_rows_here == p.b_widths[3]) mb = &tm_w3;
           }
+          load(b_dst, mb, fb, kc * BK, t.b_row, pol_w);
+          issued_mask |= 1u << s;
+          issued_par = (issued_par & ~(1u << s)) | (ph << s);
+          if (++s == p.stages) { s = 0; ph ^= 1u; }
         }
       }
       if (!ok) {
-        // Do not leave with copies in flight: wait (bounded) for the last
-        // load issued into every stage to land.
+        // Do not leave with copies in flight.  A leader (or a single CTA)
+        // waits, bounded, for the last load into every stage to land; in a
+        // pair the other CTA's loads complete on the leader's barriers, so it
+        // waits a fixed, bounded time instead.
         const uint64_t dl = globaltimer_ns() + 50000000ull;
-        for (int q = 0; q < p.stages; ++q) {
-          if (!(issued_mask >> q & 1u)) continue;
-          const uint32_t par = (issued_par >> q) & 1u;
-          while (!mbar_try_wait(full_bar(q), par) && globaltimer_ns() < dl) {
+        if (leader) {
+          for (int q = 0; q < p.stages; ++q) {
+            if (!(issued_mask >> q & 1u)) continue;
+            const uint32_t par = (issued_par >> q) & 1u;
+            while (!mbar_try_wait(full_bar(q), par) && globaltimer_ns() < dl) {
+            }
+          }
+        } else {
+          const uint64_t t_end = globaltimer_ns() + 200000ull;
+          while (globaltimer_ns() < t_end) {
           }
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------ MMA issuer ----
-    if (lane == 0) {
-      const uint32_t idesc = umma_idesc_bf16_f32(A_ROWS, p.n_mma);
+    if (lane == 0 && leader) {
       int s = 0;
       uint32_t ph = 0;
       int tb = 0;
       uint32_t tph = 0;
       bool ok = true;
-      auto do_tile = [&]() -> bool {
-        if (!mbar_wait(tempty_bar(tb), tph ^ 1u, deadline, abort_flag, p.status)) return false;
+      auto commit = [&](uint32_t bar) {
+        if (PAIR)
+          umma_commit_pair_multicast(bar, 0x3);
+        else
+          umma_commit(bar);
+      };
+      Tile t;
+      for (int k = 0; ok && get_tile<MODE, PAIR>(p, k, rank, t); ++k) {
+        const uint32_t idesc = umma_idesc_bf16_f32(PAIR ? 2 * A_ROWS : A_ROWS, t.n_cols);
+        if (!mbar_wait(tempty_bar(tb), tph ^ 1u, deadline, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(tb * p.buf_cols);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(tb * TILE_N);
         for (int kc = 0; kc < p.num_kc; ++kc) {
-          if (!mbar_wait(full_bar(s), ph, deadline, abort_flag, p.status)) return false;
+          if (!mbar_wait(full_bar(s), ph, deadline, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          const uint64_t adesc = umma_desc_sw128(sbase + L.a + s * A_STAGE_BYTES);
+          const uint64_t adesc = umma_desc_sw128(sbase + L.a + s * p.a_stage_bytes);
           const uint64_t bdesc = umma_desc_sw128(sbase + L.b + s * p.b_stage_bytes);
 #pragma unroll
-          for (int k = 0; k < BK / UMMA_K; ++k) {
-            // advance the start address by k * 32 bytes (encoded >> 4)
-            umma_bf16(d_tmem, adesc + 2ull * k, bdesc + 2ull * k, idesc, (kc | k) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+            // advance the start address by kk * 32 bytes (encoded >> 4)
+            const uint32_t acc = (kc | kk) != 0 ? 1u : 0u;
+            if (PAIR)
+              umma_bf16_pair(d_tmem, adesc + 2ull * kk, bdesc + 2ull * kk, idesc, acc);
+            else
+              umma_bf16(d_tmem, adesc + 2ull * kk, bdesc + 2ull * kk, idesc, acc);
           }
-          umma_commit(empty_bar(s));
+          commit(empty_bar(s));
           if (++s == p.stages) { s = 0; ph ^= 1u; }
         }
-        umma_commit(tfull_bar(tb));
+        if (!ok) break;
+        commit(tfull_bar(tb));
         if (++tb == 2) { tb = 0; tph ^= 1u; }
-        return true;
-      };
-      if (MODE == MODE_SWAP) {
-        for (int t0 = r0; ok && t0 < r1; t0 += A_ROWS) ok = do_tile();
-      } else {
-        int mt, vt, slot;
-        bool first, last;
-        for (int k = 0; ok && large_tile(p, k, mt, vt, slot, first, last); ++k) ok = do_tile();
       }
       // Every MMA this thread issued has completed before TMEM is released.
-      umma_commit(drain_bar);
+      if (PAIR)
+        umma_commit_pair(drain_bar);
+      else
+        umma_commit(drain_bar);
       const uint64_t dl = globaltimer_ns() + 50000000ull;
       while (!mbar_try_wait(drain_bar, 0) && globaltimer_ns() < dl) {
       }
     }
   } else {
     // ------------------------------------------------------ epilogue ------
-    const int e = threadIdx.x - 64;           // 0..127
+    const int ew = warp - 2;                  // 0..7
     const int quarter = warp & 3;             // TMEM lanes this warp may access
+    const int half = ew >> 2;                 // which half of the tile's columns
     const int trow = quarter * 32 + lane;     // accumulator row held by this thread
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     TopState st;
     st.reset();
     int tb = 0;
     uint32_t tph = 0;
-
-    if (MODE == MODE_SWAP) {
-      float* T = reinterpret_cast<float*>(smem + L.t);
-      const int g = p.g;
-      const int n = e / g;
-      const int sub = e - n * g;
-      const bool active = n < p.M;
-      const int ncols = (p.M + 15) & ~15;
-      for (int t0 = r0; t0 < r1; t0 += A_ROWS) {
-        const int rows = min(A_ROWS, r1 - t0);
-        if (e == 0) *epi_ok = mbar_wait(tfull_bar(tb), tph, deadline, abort_flag, p.status) ? 1 : 0;
-        named_barrier_sync(1, EPI_THREADS);
-        if (!*epi_ok) break;
-        tc_fence_after();
-        const uint32_t taddr = tmem_base + static_cast<uint32_t>(tb * p.buf_cols) + lane_off;
-        for (int c0 = 0; c0 < ncols; c0 += 16) {
-          float x[16];
-          tmem_ld16(taddr + c0, x);
-          tmem_ld_wait();
+    Tile t;
+    for (int k = 0; get_tile<MODE, PAIR>(p, k, rank, t); ++k) {
+      int ok = 0;
+      if (lane == 0) ok = mbar_wait(tfull_bar(tb), tph, deadline, abort_flag, p.status) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      if (t.first) st.reset();
+      const int row = t.a_row + trow;
+      const int nch = t.n_cols / 16;
+      const int split = (nch + 1) >> 1;
+      // warps whose 32 rows are all past M only hand the buffer back
+      const int ch_end = t.a_row + quarter * 32 >= p.M ? 0 : (half ? nch : split);
+      const uint32_t taddr = tmem_base + static_cast<uint32_t>(tb * TILE_N) + lane_off;
+      for (int ch = half ? split : 0; ch < ch_end; ++ch) {
+        const int c0 = ch * 16;
+        const int vbase = t.v0 + c0;
+        if (vbase >= p.V) break;
+        float x[16];
+        tmem_ld16(taddr + c0, x);
+        tmem_ld_wait();
+        const int nvalid = min(16, p.V - vbase);
+        float cmax = -INFINITY;
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj)
+          if (jj < nvalid) cmax = fmaxf(cmax, x[jj]);
+        if (cmax > st.m) {
+          st.s *= __expf(st.m - cmax);
+          st.m = cmax;
+        }
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj)
+          if (jj < nvalid) st.s += __expf(x[jj] - st.m);
+        // Candidates of this chunk that can enter the list; each lane then
+        // inserts only its own, so the warp loops max_lane(count) times.
+        uint32_t pend = 0;
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj)
+          if (jj < nvalid && x[jj] > st.v[KTOP - 1]) pend |= 1u << jj;
+        while (__any_sync(0xffffffffu, pend != 0)) {
+          if (pend) {
+            const int jj = __ffs(pend) - 1;
+            pend &= pend - 1;
+            float xv = x[0];
+#pragma unroll
+            for (int q = 1; q < 16; ++q) xv = jj == q ? x[q] : xv;
+            st.insert_scan(xv, vbase + jj);
+          }
+        }
+        if (p.z_dbg && row < p.M) {
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj)
-            if (c0 + jj < p.M) T[(c0 + jj) * p.t_stride + trow] = x[jj];
+            if (jj < nvalid) p.z_dbg[static_cast<size_t>(row) * p.V + vbase + jj] = x[jj];
         }
-        tc_fence_before();
+      }
+      // release the TMEM buffer to the MMA issuer (the leader's barrier)
+      tc_fence_before();
+      if (PAIR && !leader)
+        mbar_arrive_cluster(mapa_shared(tempty_bar(tb), 0));
+      else
         mbar_arrive(tempty_bar(tb));
-        if (++tb == 2) { tb = 0; tph ^= 1u; }
-        named_barrier_sync(1, EPI_THREADS);
-        if (active) {
-          const float* Tn = T + n * p.t_stride;
-          const int vend = min(rows, p.V - t0);
-          for (int l = sub; l < vend; l += g) {
-            const float x = Tn[l];
-            const int v = t0 + l;
-            if (p.z_dbg) p.z_dbg[static_cast<size_t>(n) * p.V + v] = x;
-            if (x > st.m) {
-              st.s = st.s * __expf(st.m - x) + 1.f;
-              st.m = x;
-            } else {
-              st.s += __expf(x - st.m);
-            }
-            st.insert(x, v);
-          }
-        }
-      }
-      // Fold the g lists of each token (g adjacent lanes) into one.
-      for (int off = 1; off < g; off <<= 1) {
-        const float m2 = __shfl_xor_sync(0xffffffffu, st.m, off);
-        const float s2 = __shfl_xor_sync(0xffffffffu, st.s, off);
-        st.merge_lse(m2, s2);
-      }
-      float ov[KTOP];
-      int oi[KTOP];
-#pragma unroll
-      for (int r = 0; r < KTOP; ++r) {
-        float bv = st.v[0];
-        int bi = st.i[0];
-        for (int off = 1; off < g; off <<= 1) {
-          const float v2 = __shfl_xor_sync(0xffffffffu, bv, off);
-          const int i2 = __shfl_xor_sync(0xffffffffu, bi, off);
-          if (better(v2, i2, bv, bi)) {
-            bv = v2;
-            bi = i2;
-          }
-        }
-        if (st.i[0] == bi && st.v[0] == bv) st.pop_head();
-        ov[r] = bv;
-        oi[r] = bi;
-      }
-      if (active && sub == 0) store_partial(p.part + static_cast<size_t>(n) * p.P + blockIdx.x, st.m, st.s, ov, oi);
-    } else {
-      int mt, vt, slot;
-      bool first, last;
-      for (int k = 0; large_tile(p, k, mt, vt, slot, first, last); ++k) {
-        int ok = 0;
-        if (lane == 0) ok = mbar_wait(tfull_bar(tb), tph, deadline, abort_flag, p.status) ? 1 : 0;
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
-        tc_fence_after();
-        if (first) st.reset();
-        const int row = mt * A_ROWS + trow;
-        const int v0 = vt * LARGE_N;
-        const uint32_t taddr = tmem_base + static_cast<uint32_t>(tb * p.buf_cols) + lane_off;
-        for (int c0 = 0; c0 < LARGE_N && v0 + c0 < p.V; c0 += 16) {
-          float x[16];
-          tmem_ld16(taddr + c0, x);
-          tmem_ld_wait();
-          const int nvalid = min(16, p.V - (v0 + c0));
-          float cmax = -INFINITY;
-#pragma unroll
-          for (int jj = 0; jj < 16; ++jj)
-            if (jj < nvalid) cmax = fmaxf(cmax, x[jj]);
-          if (cmax > st.m) {
-            st.s *= __expf(st.m - cmax);
-            st.m = cmax;
-          }
-#pragma unroll
-          for (int jj = 0; jj < 16; ++jj)
-            if (jj < nvalid) st.s += __expf(x[jj] - st.m);
-          // Candidates of this chunk that can enter the list; each lane then
-          // inserts only its own, so the warp loops max_lane(count) times.
-          uint32_t pend = 0;
-#pragma unroll
-          for (int jj = 0; jj < 16; ++jj)
-            if (jj < nvalid && x[jj] >= st.v[KTOP - 1]) pend |= 1u << jj;
-          while (__any_sync(0xffffffffu, pend != 0)) {
-            if (pend) {
-              const int jj = __ffs(pend) - 1;
-              pend &= pend - 1;
-              float xv = x[0];
-#pragma unroll
-              for (int q = 1; q < 16; ++q) xv = jj == q ? x[q] : xv;
-              st.insert(xv, v0 + c0 + jj);
-            }
-          }
-          if (p.z_dbg && row < p.M) {
-#pragma unroll
-            for (int jj = 0; jj < 16; ++jj)
-              if (jj < nvalid) p.z_dbg[static_cast<size_t>(row) * p.V + v0 + c0 + jj] = x[jj];
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(tempty_bar(tb));
-        if (++tb == 2) { tb = 0; tph ^= 1u; }
-        if (last && row < p.M) store_partial(p.part + static_cast<size_t>(row) * p.P + slot, st.m, st.s, st.v, st.i);
-      }
+      if (++tb == 2) { tb = 0; tph ^= 1u; }
+      if (t.last && row < p.M)
+        store_partial(p.part + static_cast<size_t>(row) * p.P + 2 * t.slot + half, st.m, st.s, st.v, st.i);
     }
   }
 
   pdl_trigger();
   tc_fence_before();
   __syncthreads();
+  __syncwarp();
+  if (PAIR) cluster_sync_all();  // the pair's MMAs and remote arrivals are done
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, p.tmem_cols);
+    if (PAIR)
+      tmem_dealloc_pair(tmem_base, p.tmem_cols);
+    else
+      tmem_dealloc(tmem_base, p.tmem_cols);
   }
 }
 
-// One warp per row: fold P partial records into the final top-16 and lse.
-__global__ void __launch_bounds__(128) merge_kernel(const Partial* __restrict__ part, int M, int P,
-                                                    float* __restrict__ topk_logp,
-                                                    int32_t* __restrict__ topk_idx,
-                                                    float* __restrict__ lse) {
-  const int lane = threadIdx.x & 31;
-  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  pdl_wait();
-  pdl_trigger();
-  if (row >= M) return;
-  TopState st;
-  st.reset();
-  const Partial* base = part + static_cast<size_t>(row) * P;
-  // Records are loaded one ahead so the next load overlaps this record's work.
-  PartialRegs cur, nxt;
-  if (lane < P) cur.load(base + lane);
-  for (int q = lane; q < P; q += 32) {
-    if (q + 32 < P) nxt.load(base + q + 32);
-    st.merge_lse(cur.m(), cur.s());
-    float rv[KTOP];
-    int ri[KTOP];
-    cur.lists(rv, ri);
-    st.insert_sorted(rv, ri);
-    cur = nxt;
-  }
+// Fold a warp's 32 lists (one per lane, plus each lane's (max, sum exp)) into
+// one: afterwards lane r < 16 holds entry r of the merged list and every lane
+// holds the merged (m, s).
+__device__ __forceinline__ void warp_merge(TopState& st, float& out_v, int& out_i) {
   for (int off = 1; off < 32; off <<= 1) {
     const float m2 = __shfl_xor_sync(0xffffffffu, st.m, off);
     const float s2 = __shfl_xor_sync(0xffffffffu, st.s, off);
     st.merge_lse(m2, s2);
   }
-  const float row_lse = st.m + logf(st.s);
-  float my_v = 0.f;
-  int my_i = 0;
+  const int lane = threadIdx.x & 31;
+  out_v = -INFINITY;
+  out_i = 0x7fffffff;
 #pragma unroll
   for (int r = 0; r < KTOP; ++r) {
     float bv = st.v[0];
@@ -491,13 +496,95 @@ __global__ void __launch_bounds__(128) merge_kernel(const Partial* __restrict__ 
     }
     if (st.i[0] == bi && st.v[0] == bv) st.pop_head();
     if (lane == r) {
-      my_v = bv;
-      my_i = bi;
+      out_v = bv;
+      out_i = bi;
     }
   }
+}
+
+// Fold a lane's share of a row's partial records (q = first, first+step, ...)
+// into its list; records are loaded one ahead so loads overlap the work.
+__device__ __forceinline__ void fold_records(TopState& st, const Partial* base, int first, int step, int P) {
+  PartialRegs cur, nxt;
+  if (first < P) cur.load(base + first);
+  for (int q = first; q < P; q += step) {
+    if (q + step < P) nxt.load(base + q + step);
+    st.merge_lse(cur.m(), cur.s());
+    float rv[KTOP];
+    int ri[KTOP];
+    cur.lists(rv, ri);
+    st.insert_sorted(rv, ri);
+    cur = nxt;
+  }
+}
+
+// Few records per row: one warp per row.
+__global__ void __launch_bounds__(128) merge_kernel(const Partial* __restrict__ part, int M, int P,
+                                                    float* __restrict__ topk_logp,
+                                                    int32_t* __restrict__ topk_idx,
+                                                    float* __restrict__ lse) {
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  pdl_wait();
+  pdl_trigger();
+  if (row >= M) return;
+  TopState st;
+  st.reset();
+  fold_records(st, part + static_cast<size_t>(row) * P, lane, 32, P);
+  float v;
+  int ix;
+  warp_merge(st, v, ix);
+  const float row_lse = st.m + logf(st.s);
   if (lane < KTOP) {
-    topk_logp[static_cast<size_t>(row) * KTOP + lane] = my_v - row_lse;
-    topk_idx[static_cast<size_t>(row) * KTOP + lane] = my_i;
+    topk_logp[static_cast<size_t>(row) * KTOP + lane] = v - row_lse;
+    topk_idx[static_cast<size_t>(row) * KTOP + lane] = ix;
+  }
+  if (lane == 0 && lse != nullptr) lse[row] = row_lse;
+}
+
+// Many records per row: one CTA of 256 threads per row; eight warp lists are
+// merged again by warp 0.
+__global__ void __launch_bounds__(256) merge_kernel_wide(const Partial* __restrict__ part, int M, int P,
+                                                         float* __restrict__ topk_logp,
+                                                         int32_t* __restrict__ topk_idx,
+                                                         float* __restrict__ lse) {
+  __shared__ float sv[8][KTOP];
+  __shared__ int si[8][KTOP];
+  __shared__ float sm[8], ss[8];
+  const int lane = threadIdx.x & 31;
+  const int w = threadIdx.x >> 5;
+  const int row = blockIdx.x;
+  pdl_wait();
+  pdl_trigger();
+  TopState st;
+  st.reset();
+  fold_records(st, part + static_cast<size_t>(row) * P, threadIdx.x, blockDim.x, P);
+  float v;
+  int ix;
+  warp_merge(st, v, ix);
+  if (lane < KTOP) {
+    sv[w][lane] = v;
+    si[w][lane] = ix;
+  }
+  if (lane == 0) {
+    sm[w] = st.m;
+    ss[w] = st.s;
+  }
+  __syncthreads();
+  if (w != 0) return;
+  TopState fin;
+  fin.reset();
+  if (lane < 8) fin.merge_lse(sm[lane], ss[lane]);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int c = q * 32 + lane;  // candidate c of the 8 x 16 warp lists
+    fin.insert(sv[c >> 4][c & 15], si[c >> 4][c & 15]);
+  }
+  warp_merge(fin, v, ix);
+  const float row_lse = fin.m + logf(fin.s);
+  if (lane < KTOP) {
+    topk_logp[static_cast<size_t>(row) * KTOP + lane] = v - row_lse;
+    topk_idx[static_cast<size_t>(row) * KTOP + lane] = ix;
   }
   if (lane == 0 && lse != nullptr) lse[row] = row_lse;
 }
@@ -519,6 +606,12 @@ static unsigned long long timeout_ns_from_env() {
     return static_cast<unsigned long long>(ms) * 1000000ull;
   }();
   return v;
+}
+
+// Pairs (2-CTA MMA) are used unless DFLASH_PAIR=0 (read at every call).
+static bool pair_allowed() {
+  const char* e = std::getenv("DFLASH_PAIR");
+  return !(e != nullptr && e[0] == '0');
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -551,12 +644,60 @@ static bool make_map(CUtensorMap* m, const void* base, int rows, int cols, int b
   return r == CUDA_SUCCESS;
 }
 
+template <int MODE, bool PAIR>
+static cudaError_t set_smem_attr() {
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    err = cudaFuncSetAttribute(lmhead_kernel<MODE, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SMEM_BUDGET + 2048);
+  });
+  return err;
+}
+
+// Clusters of two that can be resident at once (0 when pairs cannot run).
+template <int MODE>
+static int max_pair_clusters() {
+  static std::once_flag once;
+  static int n = 0;
+  std::call_once(once, [] {
+    if (set_smem_attr<MODE, true>() != cudaSuccess) return;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = SMEM_BUDGET + 1024;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int c = 0;
+    if (cudaOccupancyMaxActiveClusters(&c, lmhead_kernel<MODE, true>, &cfg) == cudaSuccess) n = c;
+    cudaGetLastError();
+  });
+  return n;
+}
+
 struct Plan {
   int mode;
+  bool pair;
   int grid;
   Params p;
   size_t smem;
 };
+
+// Deepest ring of `per_stage` bytes that fits the shared-memory budget.
+static int fit_stages(Params& p, int cap) {
+  int best = 0;
+  for (int s = 2; s <= cap; ++s) {
+    p.stages = s;
+    if (smem_layout(p).total + 1024 <= static_cast<uint32_t>(SMEM_BUDGET)) best = s;
+  }
+  p.stages = best;
+  return best;
+}
 
 static bool make_plan(int M, int V, int d, int sms, Plan& pl) {
   if (M < 1 || V < 16 || d < 8 || d % 8 != 0 || sms < 1) return false;
@@ -566,58 +707,86 @@ static bool make_plan(int M, int V, int d, int sms, Plan& pl) {
   p.V = V;
   p.d = d;
   p.num_kc = (d + BK - 1) / BK;
-  if (M <= 128) {
-    pl.mode = MODE_SWAP;
-    p.n_mma = (M + 15) & ~15;
-    p.buf_cols = p.n_mma;
-    int cols = 32;
-    while (cols < 2 * p.n_mma) cols <<= 1;
-    p.tmem_cols = cols;
-    p.b_stage_bytes = p.n_mma * BK * 2;
-    p.b_tx_bytes = p.b_stage_bytes;
+  p.tmem_cols = 2 * TILE_N;
+  if (M <= A_ROWS) {
+    pl.mode = MODE_STREAM;
+    pl.pair = false;
+    p.a_box = (M + 15) & ~15;
+    p.a_stage_bytes = p.a_box * BK * 2;
+    p.b_rows = TILE_N;
+    p.b_stage_bytes = p.b_rows * BK * 2;
     p.units = (V + 15) / 16;
-    int g = 32;
-    while (g > 1 && g * M > EPI_THREADS) g >>= 1;
-    p.g = g;
-    p.t_stride = 128 + g;
-    p.t_bytes = ((M * p.t_stride * 4) + 1023) & ~1023;
     pl.grid = p.units < sms ? p.units : sms;
-    p.P = pl.grid;
-    const int fixed = p.t_bytes + 1024 + 512;
-    int stages = (SMEM_BUDGET - fixed) / (A_STAGE_BYTES + p.b_stage_bytes);
-    if (stages > 16) stages = 16;
-    if (stages < 2) return false;
-    p.stages = stages;
+    p.P = 2 * pl.grid;
+    // the widths STREAM tiles can take (see get_tile): per unit count u, the
+    // main width 16*ceil(u/nt) and the last tile's remainder
+    int nw = 0;
+    for (int j = 0; j < 4; ++j) p.b_widths[j] = -1;
+    const int u_lo = p.units / pl.grid;
+    for (int u = u_lo; u <= u_lo + 1; ++u) {
+      if (u < 1) continue;
+      const int nt = (u + TILE_N / 16 - 1) / (TILE_N / 16);
+      const int wu = (u + nt - 1) / nt;
+      const int ws[2] = {16 * wu, 16 * (u - (nt - 1) * wu)};
+      for (int w : ws) {
+        if (w <= 0) continue;
+        bool have = false;
+        for (int j = 0; j < nw; ++j) have = have || p.b_widths[j] == w;
+        if (!have) {
+          if (nw == 4) return false;
+          p.b_widths[nw++] = w;
+        }
+      }
+    }
+    if (fit_stages(p, 12) < 2) return false;
   } else {
     pl.mode = MODE_LARGE;
-    p.n_mma = LARGE_N;
-    p.buf_cols = LARGE_N;
-    p.tmem_cols = 512;
-    p.b_stage_bytes = LARGE_N * BK * 2;
-    p.b_tx_bytes = p.b_stage_bytes;
-    p.g = 1;
-    p.t_stride = 0;
-    p.t_bytes = 0;
-    p.m_tiles = (M + A_ROWS - 1) / A_ROWS;
-    p.v_tiles = (V + LARGE_N - 1) / LARGE_N;
-    const long long tiles = static_cast<long long>(p.m_tiles) * p.v_tiles;
-    const int g_str = static_cast<int>(tiles < sms ? tiles : sms);
-    const long long t_str = (tiles + g_str - 1) / g_str;           // tiles on the busiest CTA
-    int nr = sms / p.m_tiles;
+    const int clusters = pair_allowed() ? max_pair_clusters<MODE_LARGE>() : 0;
+    pl.pair = clusters >= 1;
+    p.a_box = A_ROWS;
+    p.a_stage_bytes = A_ROWS * BK * 2;
+    p.b_rows = pl.pair ? TILE_N / 2 : TILE_N;
+    p.b_stage_bytes = p.b_rows * BK * 2;
+    const int m_rows = pl.pair ? 2 * A_ROWS : A_ROWS;
+    p.m_tiles = (M + m_rows - 1) / m_rows;
+    p.v_tiles = (V + TILE_N - 1) / TILE_N;
+    const int units = pl.pair ? (clusters < sms / 2 ? clusters : sms / 2) : sms;
+    // cost = tiles on the busiest unit, with each job restart charged as a
+    // fraction of a tile (its candidate list starts empty)
+    const double restart = 0.15;
+    double best = 1e30;
+    int used = 1;
+    int nr = units / p.m_tiles;
     if (nr > p.v_tiles) nr = p.v_tiles;
-    const long long t_run = nr >= 1 ? (p.v_tiles + nr - 1) / nr : (1ll << 40);
-    if (t_run <= t_str) {
-      p.sched = SCHED_RUNS;
-      p.nr = nr;
-      pl.grid = nr * p.m_tiles;
-      p.P = nr;
-    } else {
-      p.sched = SCHED_STRIDED;
-      p.nr = 0;
-      pl.grid = g_str;
-      p.P = p.v_tiles;
+    if (nr >= 1) {
+      const long long t_run = (p.v_tiles + nr - 1) / nr;
+      const double c = t_run * (1.0 + restart / t_run);
+      if (c < best) {
+        best = c;
+        p.sched = SCHED_RUNS;
+        p.nr = nr;
+        used = nr * p.m_tiles;
+        p.P = 2 * nr;
+      }
     }
-    p.stages = 4;
+    for (int R = 1; R <= 64; R *= 2) {
+      const int nvb = (p.v_tiles + R - 1) / R;
+      const long long jobs = static_cast<long long>(p.m_tiles) * nvb;
+      const int u = static_cast<int>(jobs < units ? jobs : units);
+      const long long t_blk = ((jobs + u - 1) / u) * R;
+      const double c = t_blk * (1.0 + restart / R);
+      if (c < best) {
+        best = c;
+        p.sched = SCHED_BLOCKS;
+        p.R = R;
+        p.n_vblocks = nvb;
+        p.nr = 0;
+        used = u;
+        p.P = 2 * nvb;
+      }
+    }
+    pl.grid = pl.pair ? 2 * used : used;
+    if (fit_stages(p, 8) < 2) return false;
   }
   pl.smem = smem_layout(p).total + 1024;
   return true;
@@ -625,6 +794,14 @@ static bool make_plan(int M, int V, int d, int sms, Plan& pl) {
 
 static size_t part_bytes(const Plan& pl) {
   return static_cast<size_t>(pl.p.M) * pl.p.P * sizeof(Partial);
+}
+
+template <int MODE, bool PAIR>
+static cudaError_t launch_main(const Plan& pl, const CUtensorMap& ta, const CUtensorMap* tb, cudaStream_t st) {
+  const cudaError_t e = set_smem_attr<MODE, PAIR>();
+  if (e != cudaSuccess) return e;
+  return launch_kernel_cluster(lmhead_kernel<MODE, PAIR>, dim3(pl.grid), dim3(NUM_THREADS), pl.smem, st,
+                               PAIR ? 2 : 1, ta, tb[0], tb[1], tb[2], tb[3], pl.p);
 }
 
 static int launch(const dflash_bf16* H, const dflash_bf16* W, int M, int V, int d, float* topk_logp,
@@ -643,44 +820,36 @@ static int launch(const dflash_bf16* H, const dflash_bf16* W, int M, int V, int 
   p.status = dev_status;
   p.timeout_ns = timeout_ns_from_env();
 
-  CUtensorMap ta, ta16, tb;
-  bool ok;
-  if (pl.mode == MODE_SWAP) {
-    ok = make_map(&ta, W, V, d, A_ROWS) && make_map(&ta16, W, V, d, 16) && make_map(&tb, H, M, d, p.n_mma);
-  } else {
-    ok = make_map(&ta, H, M, d, A_ROWS) && make_map(&tb, W, V, d, LARGE_N);
-    ta16 = ta;
+  // W maps: the full tile box, then (STREAM) one box per other tile width
+  CUtensorMap ta, tb[4];
+  bool ok = make_map(&ta, H, M, d, p.a_box) &&
+            make_map(&tb[0], W, V, d, pl.mode == MODE_STREAM ? p.b_widths[0] : p.b_rows);
+  for (int j = 1; j < 4; ++j) {
+    if (pl.mode == MODE_STREAM && p.b_widths[j] > 0)
+      ok = ok && make_map(&tb[j], W, V, d, p.b_widths[j]);
+    else
+      tb[j] = tb[0];
   }
   if (!ok) return DFLASH_ERR_CUDA;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  static std::once_flag once[2];
-  static cudaError_t attr_err[2] = {cudaSuccess, cudaSuccess};
-  if (pl.mode == MODE_SWAP) {
-    std::call_once(once[0], [] {
-      attr_err[0] = cudaFuncSetAttribute(lmhead_kernel<MODE_SWAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         SMEM_BUDGET + 2048);
-    });
-    if (attr_err[0] != cudaSuccess) return DFLASH_ERR_CUDA;
-    if (launch_kernel(lmhead_kernel<MODE_SWAP>, dim3(pl.grid), dim3(NUM_THREADS), pl.smem, st, ta, ta16, tb, p) !=
-        cudaSuccess)
-      return DFLASH_ERR_CUDA;
-  } else {
-    std::call_once(once[1], [] {
-      attr_err[1] = cudaFuncSetAttribute(lmhead_kernel<MODE_LARGE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         SMEM_BUDGET + 2048);
-    });
-    if (attr_err[1] != cudaSuccess) return DFLASH_ERR_CUDA;
-    if (launch_kernel(lmhead_kernel<MODE_LARGE>, dim3(pl.grid), dim3(NUM_THREADS), pl.smem, st, ta, ta16, tb, p) !=
-        cudaSuccess)
-      return DFLASH_ERR_CUDA;
-  }
-  if (cudaGetLastError() != cudaSuccess) return DFLASH_ERR_CUDA;
+  cudaError_t e;
+  if (pl.mode == MODE_STREAM)
+    e = launch_main<MODE_STREAM, false>(pl, ta, tb, st);
+  else
+    e = pl.pair ? launch_main<MODE_LARGE, true>(pl, ta, tb, st) : launch_main<MODE_LARGE, false>(pl, ta, tb, st);
+  if (e != cudaSuccess) return DFLASH_ERR_CUDA;
   if (z_dbg == nullptr) {
-    const int rows_per_cta = 4;
-    if (launch_kernel(merge_kernel, dim3((M + rows_per_cta - 1) / rows_per_cta), dim3(32 * rows_per_cta), 0, st,
-                      static_cast<const Partial*>(p.part), M, p.P, topk_logp, topk_idx, lse) != cudaSuccess)
-      return DFLASH_ERR_CUDA;
+    const Partial* part = p.part;
+    cudaError_t me;
+    if (p.P >= 64) {
+      me = launch_kernel(merge_kernel_wide, dim3(M), dim3(256), 0, st, part, M, p.P, topk_logp, topk_idx, lse);
+    } else {
+      const int rows_per_cta = 4;
+      me = launch_kernel(merge_kernel, dim3((M + rows_per_cta - 1) / rows_per_cta), dim3(32 * rows_per_cta), 0, st,
+                         part, M, p.P, topk_logp, topk_idx, lse);
+    }
+    if (me != cudaSuccess) return DFLASH_ERR_CUDA;
   }
   return DFLASH_OK;
 }

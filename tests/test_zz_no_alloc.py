@@ -95,8 +95,9 @@ def test_static_matches_workspace_version_two_calls_in_a_row():
 
 def test_static_rejects_sizes_beyond_the_array():
     lib = _lib()
-    M, V, d = 4096, 129280, 4096          # needs far more than DFLASH_STATIC_SCRATCH_BYTES
-    assert lib.dflash_lmhead_topk_workspace(M, V, d) > (8 << 20)
+    # a shape whose partial records need far more than DFLASH_STATIC_SCRATCH_BYTES
+    M, V, d = next((m, v, dd) for m, v, dd in [(10240, 151936, 4096), (20480, 151936, 4096), (40960, 262144, 1024)]
+                   if lib.dflash_lmhead_topk_workspace(m, v, dd) > (8 << 20))
     fake = ctypes.c_void_p(0x1000)        # never dereferenced: rejected on the host
     rc = lib.dflash_lmhead_topk_static(fake, fake, M, V, d, 16, fake, fake, None, None, None)
     assert rc == 2

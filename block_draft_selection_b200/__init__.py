@@ -13,6 +13,8 @@ from ._binding import (  # noqa: F401
     K_TOP,
     LIB_PATH,
     dflash_conv2tap,
+    dflash_conv2tap_dynamic,
+    dflash_gemm_bf16,
     dflash_lmhead_logits_debug,
     dflash_lmhead_topk,
     dflash_lmhead_topk_workspace,

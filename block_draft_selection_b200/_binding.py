@@ -49,6 +49,9 @@ def _load():
         "dflash_verify": (i32, [vp, vp, i32, i32, vp, vp, vp]),
         "dflash_select_verify": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]),
         "dflash_lmhead_topk_static": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]),
+        "dflash_gemm_bf16": (i32, [vp, vp, vp, i32, i32, i32, vp]),
+        "dflash_conv2tap_dynamic_workspace": (sz, [i32, i32, i32]),
+        "dflash_conv2tap_dynamic": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -108,6 +111,41 @@ def dflash_conv2tap(x, a0, a1, prev=None, y=None, stream=None):
     y = _out(y, "y", torch.bfloat16, (B, P, d), x.device)
     _check("dflash_conv2tap", lib.dflash_conv2tap(_ptr(x), _ptr(prev), _ptr(a0), _ptr(a1), _ptr(y),
                                                   B, P, d, _stream(stream)))
+    return y
+
+
+def dflash_gemm_bf16(A, B, C=None, stream=None):
+    """C [M,N] fp32 = A [M,K] bf16 . B [N,K]^T, on the tensor-core path."""
+    _need(A, "A", torch.bfloat16)
+    _need(B, "B", torch.bfloat16)
+    M, K = A.shape
+    N = B.shape[0]
+    if B.shape[1] != K:
+        raise ValueError("A and B disagree on K")
+    C = _out(C, "C", torch.float32, (M, N), A.device)
+    _check("dflash_gemm_bf16", lib.dflash_gemm_bf16(_ptr(A), _ptr(B), _ptr(C), M, N, K, _stream(stream)))
+    return C
+
+
+def dflash_conv2tap_dynamic(x, a0, a1, wc, prev=None, y=None, ws=None, stream=None):
+    """Two-tap conv with per-16-channel tap corrections delta = x . Wc^T.
+    x [B,P,d], a0/a1 [d], wc [2*d/16, d], prev [B,d] or None: bf16."""
+    _need(x, "x", torch.bfloat16)
+    B, P, d = x.shape
+    _need(a0, "a0", torch.bfloat16, (d,))
+    _need(a1, "a1", torch.bfloat16, (d,))
+    _need(wc, "wc", torch.bfloat16, (2 * (d // 16), d))
+    if prev is not None:
+        _need(prev, "prev", torch.bfloat16, (B, d))
+    y = _out(y, "y", torch.bfloat16, (B, P, d), x.device)
+    if ws is None:
+        n = int(lib.dflash_conv2tap_dynamic_workspace(B, P, d))
+        if n == 0:
+            raise DFlashError("dflash_conv2tap_dynamic_workspace", DFLASH_ERR_INVALID_ARG)
+        ws = torch.empty(n, dtype=torch.uint8, device=x.device)
+    _check("dflash_conv2tap_dynamic", lib.dflash_conv2tap_dynamic(
+        _ptr(x), _ptr(prev), _ptr(a0), _ptr(a1), _ptr(wc), _ptr(y), B, P, d, _ptr(ws), ws.numel(),
+        _stream(stream)))
     return y
 
 

@@ -85,6 +85,8 @@ struct Params {
   int R;             // BLOCKS: vocabulary tiles per job
   int n_vblocks;     // BLOCKS: ceil(v_tiles / R)
   int b_widths[4];   // STREAM: the tile widths, one tensor map each
+  int merge_halves;  // one run per unit: the two column halves merge in-kernel
+  int store_only;    // plain GEMM: write z to z_dbg, no log-softmax / top-16
   // outputs
   Partial* part;     // [M][P]
   int P;
@@ -388,6 +390,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     st.reset();
     int tb = 0;
     uint32_t tph = 0;
+    int run_slot = -1;   // merge_halves: slot of the completed run
+    int run_row = p.M;   // merge_halves: this thread's token row in that run
     Tile t;
     for (int k = 0; get_tile<MODE, PAIR>(p, k, rank, t); ++k) {
       int ok = 0;
@@ -410,6 +414,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_ld16(taddr + c0, x);
         tmem_ld_wait();
         const int nvalid = min(16, p.V - vbase);
+        if (p.store_only) {
+          if (row < p.M) {
+            float* zr = p.z_dbg + static_cast<size_t>(row) * p.V + vbase;
+            if (nvalid == 16 && (p.V & 3) == 0) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                reinterpret_cast<float4*>(zr)[q] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+            } else {
+#pragma unroll
+              for (int jj = 0; jj < 16; ++jj)
+                if (jj < nvalid) zr[jj] = x[jj];
+            }
+          }
+          continue;
+        }
         float cmax = -INFINITY;
 #pragma unroll
         for (int jj = 0; jj < 16; ++jj)
@@ -450,8 +469,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       else
         mbar_arrive(tempty_bar(tb));
       if (++tb == 2) { tb = 0; tph ^= 1u; }
-      if (t.last && row < p.M)
-        store_partial(p.part + static_cast<size_t>(row) * p.P + 2 * t.slot + half, st.m, st.s, st.v, st.i);
+      if (t.last && !p.store_only) {
+        if (p.merge_halves) {
+          run_slot = t.slot;
+          run_row = row;
+        } else if (row < p.M)
+          store_partial(p.part + static_cast<size_t>(row) * p.P + 2 * t.slot + half, st.m, st.s, st.v, st.i);
+      }
+    }
+    if (p.merge_halves && !p.store_only) {
+      // One run per unit: its pipeline has drained, so the B stages hold the
+      // exchange.  The half-1 warp of each lane quarter publishes its lists,
+      // the half-0 warp folds them into its own and writes one record.
+      float* xs = reinterpret_cast<float*>(smem + L.b) + trow * 36;
+      if (half == 1) {
+        xs[0] = st.m;
+        xs[1] = st.s;
+#pragma unroll
+        for (int k = 0; k < KTOP; ++k) {
+          xs[2 + k] = st.v[k];
+          xs[18 + k] = __int_as_float(st.i[k]);
+        }
+      }
+      named_barrier_sync(1 + quarter, 64);
+      if (half == 0 && run_slot >= 0 && run_row < p.M) {
+        float ov[KTOP];
+        int oi[KTOP];
+#pragma unroll
+        for (int k = 0; k < KTOP; ++k) {
+          ov[k] = xs[2 + k];
+          oi[k] = __float_as_int(xs[18 + k]);
+        }
+        st.merge_lse(xs[0], xs[1]);
+        st.insert_sorted(ov, oi);
+        store_partial(p.part + static_cast<size_t>(run_row) * p.P + run_slot, st.m, st.s, st.v, st.i);
+      }
     }
   }
 
@@ -472,32 +524,54 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 // Fold a warp's 32 lists (one per lane, plus each lane's (max, sum exp)) into
 // one: afterwards lane r < 16 holds entry r of the merged list and every lane
-// holds the merged (m, s).
+// holds the merged (m, s).  Five butterfly levels; at each, a lane takes its
+// xor-partner's sorted list, keeps the 16 best of the two (the elementwise
+// better of a[k] and b[15-k], a bitonic sequence) and re-sorts them with four
+// half-cleaner stages.
+__device__ __forceinline__ void ce_desc(float& va, int& ia, float& vb, int& ib) {
+  const bool sw = better(vb, ib, va, ia);
+  const float tv = va;
+  const int ti = ia;
+  va = sw ? vb : va;
+  ia = sw ? ib : ia;
+  vb = sw ? tv : vb;
+  ib = sw ? ti : ib;
+}
+
 __device__ __forceinline__ void warp_merge(TopState& st, float& out_v, int& out_i) {
+#pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
     const float m2 = __shfl_xor_sync(0xffffffffu, st.m, off);
     const float s2 = __shfl_xor_sync(0xffffffffu, st.s, off);
     st.merge_lse(m2, s2);
+    float pv[KTOP];
+    int pi[KTOP];
+#pragma unroll
+    for (int k = 0; k < KTOP; ++k) {
+      pv[k] = __shfl_xor_sync(0xffffffffu, st.v[k], off);
+      pi[k] = __shfl_xor_sync(0xffffffffu, st.i[k], off);
+    }
+#pragma unroll
+    for (int k = 0; k < KTOP; ++k) {
+      const bool take = better(pv[KTOP - 1 - k], pi[KTOP - 1 - k], st.v[k], st.i[k]);
+      st.v[k] = take ? pv[KTOP - 1 - k] : st.v[k];
+      st.i[k] = take ? pi[KTOP - 1 - k] : st.i[k];
+    }
+#pragma unroll
+    for (int j = KTOP / 2; j >= 1; j >>= 1) {
+#pragma unroll
+      for (int k = 0; k < KTOP; ++k)
+        if ((k & j) == 0) ce_desc(st.v[k], st.i[k], st.v[k + j], st.i[k + j]);
+    }
   }
   const int lane = threadIdx.x & 31;
   out_v = -INFINITY;
   out_i = 0x7fffffff;
 #pragma unroll
   for (int r = 0; r < KTOP; ++r) {
-    float bv = st.v[0];
-    int bi = st.i[0];
-    for (int off = 1; off < 32; off <<= 1) {
-      const float v2 = __shfl_xor_sync(0xffffffffu, bv, off);
-      const int i2 = __shfl_xor_sync(0xffffffffu, bi, off);
-      if (better(v2, i2, bv, bi)) {
-        bv = v2;
-        bi = i2;
-      }
-    }
-    if (st.i[0] == bi && st.v[0] == bv) st.pop_head();
     if (lane == r) {
-      out_v = bv;
-      out_i = bi;
+      out_v = st.v[r];
+      out_i = st.i[r];
     }
   }
 }
@@ -505,9 +579,16 @@ __device__ __forceinline__ void warp_merge(TopState& st, float& out_v, int& out_
 // Fold a lane's share of a row's partial records (q = first, first+step, ...)
 // into its list; records are loaded one ahead so loads overlap the work.
 __device__ __forceinline__ void fold_records(TopState& st, const Partial* base, int first, int step, int P) {
+  if (first >= P) return;
   PartialRegs cur, nxt;
-  if (first < P) cur.load(base + first);
-  for (int q = first; q < P; q += step) {
+  cur.load(base + first);
+  if (first + step < P) nxt.load(base + first + step);
+  // the first record is already a sorted list: it becomes the starting state
+  st.m = cur.m();
+  st.s = cur.s();
+  cur.lists(st.v, st.i);
+  cur = nxt;
+  for (int q = first + step; q < P; q += step) {
     if (q + step < P) nxt.load(base + q + step);
     st.merge_lse(cur.m(), cur.s());
     float rv[KTOP];
@@ -534,7 +615,9 @@ __global__ void __launch_bounds__(128) merge_kernel(const Partial* __restrict__ 
   float v;
   int ix;
   warp_merge(st, v, ix);
-  const float row_lse = st.m + logf(st.s);
+  // one lane's lse for every slot: the butterfly leaves lanes' (m, s) equal
+  // only up to rounding, which could reorder log-probs of near-equal logits
+  const float row_lse = __shfl_sync(0xffffffffu, st.m + logf(st.s), 0);
   if (lane < KTOP) {
     topk_logp[static_cast<size_t>(row) * KTOP + lane] = v - row_lse;
     topk_idx[static_cast<size_t>(row) * KTOP + lane] = ix;
@@ -581,7 +664,7 @@ __global__ void __launch_bounds__(256) merge_kernel_wide(const Partial* __restri
     fin.insert(sv[c >> 4][c & 15], si[c >> 4][c & 15]);
   }
   warp_merge(fin, v, ix);
-  const float row_lse = fin.m + logf(fin.s);
+  const float row_lse = __shfl_sync(0xffffffffu, fin.m + logf(fin.s), 0);
   if (lane < KTOP) {
     topk_logp[static_cast<size_t>(row) * KTOP + lane] = v - row_lse;
     topk_idx[static_cast<size_t>(row) * KTOP + lane] = ix;
@@ -717,7 +800,8 @@ static bool make_plan(int M, int V, int d, int sms, Plan& pl) {
     p.b_stage_bytes = p.b_rows * BK * 2;
     p.units = (V + 15) / 16;
     pl.grid = p.units < sms ? p.units : sms;
-    p.P = 2 * pl.grid;
+    p.merge_halves = 1;
+    p.P = pl.grid;
     // the widths STREAM tiles can take (see get_tile): per unit count u, the
     // main width 16*ceil(u/nt) and the last tile's remainder
     int nw = 0;
@@ -766,7 +850,8 @@ static bool make_plan(int M, int V, int d, int sms, Plan& pl) {
         p.sched = SCHED_RUNS;
         p.nr = nr;
         used = nr * p.m_tiles;
-        p.P = 2 * nr;
+        p.merge_halves = 1;
+        p.P = nr;
       }
     }
     for (int R = 1; R <= 64; R *= 2) {
@@ -782,6 +867,7 @@ static bool make_plan(int M, int V, int d, int sms, Plan& pl) {
         p.n_vblocks = nvb;
         p.nr = 0;
         used = u;
+        p.merge_halves = 0;
         p.P = 2 * nvb;
       }
     }
@@ -806,16 +892,17 @@ static cudaError_t launch_main(const Plan& pl, const CUtensorMap& ta, const CUte
 
 static int launch(const dflash_bf16* H, const dflash_bf16* W, int M, int V, int d, float* topk_logp,
                   int32_t* topk_idx, float* lse, float* z_dbg, void* ws, size_t ws_bytes, int* dev_status,
-                  void* stream) {
-  if (!H || !W || !ws) return DFLASH_ERR_INVALID_ARG;
+                  void* stream, bool store_only = false) {
+  if (!H || !W || (!ws && !store_only)) return DFLASH_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(H) & 15) || (reinterpret_cast<uintptr_t>(W) & 15) ||
-      (reinterpret_cast<uintptr_t>(ws) & 255))
+      (reinterpret_cast<uintptr_t>(ws) & 255) || (store_only && (reinterpret_cast<uintptr_t>(z_dbg) & 15)))
     return DFLASH_ERR_INVALID_ARG;
   Plan pl;
   if (!make_plan(M, V, d, num_sms_current(), pl)) return DFLASH_ERR_INVALID_ARG;
-  if (ws_bytes < part_bytes(pl)) return DFLASH_ERR_WORKSPACE;
+  if (!store_only && ws_bytes < part_bytes(pl)) return DFLASH_ERR_WORKSPACE;
   Params& p = pl.p;
   p.part = static_cast<Partial*>(ws);
+  p.store_only = store_only ? 1 : 0;
   p.z_dbg = z_dbg;
   p.status = dev_status;
   p.timeout_ns = timeout_ns_from_env();
@@ -839,7 +926,7 @@ static int launch(const dflash_bf16* H, const dflash_bf16* W, int M, int V, int 
   else
     e = pl.pair ? launch_main<MODE_LARGE, true>(pl, ta, tb, st) : launch_main<MODE_LARGE, false>(pl, ta, tb, st);
   if (e != cudaSuccess) return DFLASH_ERR_CUDA;
-  if (z_dbg == nullptr) {
+  if (z_dbg == nullptr && !store_only) {
     const Partial* part = p.part;
     cudaError_t me;
     if (p.P >= 64) {
@@ -874,6 +961,12 @@ extern "C" int dflash_lmhead_logits_debug(const dflash_bf16* H, const dflash_bf1
                                           float* z, void* ws, size_t ws_bytes, int* dev_status, void* stream) {
   if (!z) return DFLASH_ERR_INVALID_ARG;
   return dflash::lm::launch(H, W, M, V, d, nullptr, nullptr, nullptr, z, ws, ws_bytes, dev_status, stream);
+}
+
+extern "C" int dflash_gemm_bf16(const dflash_bf16* A, const dflash_bf16* B, float* C, int M, int N, int K,
+                                void* stream) {
+  if (!C || N < 16) return DFLASH_ERR_INVALID_ARG;
+  return dflash::lm::launch(A, B, M, N, K, nullptr, nullptr, nullptr, C, nullptr, 0, nullptr, stream, true);
 }
 
 // ---------------------------------------------------------------------------

@@ -26,7 +26,7 @@ K_TOP = 16
 
 # Order of the per-array child streams; fixed so every array is reproducible.
 STREAMS = ("H", "W", "a0", "a1", "x_conv", "prev", "E", "M", "noise", "bonus",
-           "topk", "verify")
+           "topk", "verify", "Wc", "gate")
 
 
 @dataclasses.dataclass(frozen=True)
@@ -134,6 +134,14 @@ def conv_input(w: Workload):
     x = _normal_bf16(rng_for(w.seed, "x_conv"), (w.B, w.P, w.d), 1.0)
     prev = _normal_bf16(rng_for(w.seed, "prev"), (w.B, w.d), 1.0)
     return x, prev
+
+
+def conv_correction(w: Workload, scale: float = 0.05) -> np.ndarray:
+    """Dynamic-conv correction projection Wc [2*d/16, d] bf16: rows 0..d/16-1
+    map the hidden state to tap-0 corrections of the 16-channel groups, the
+    rest to tap-1 corrections.  N(0, (scale^2)/d), so a correction is about
+    N(0, scale^2) for unit-variance inputs ("a small correction")."""
+    return _normal_bf16(rng_for(w.seed, "Wc"), (2 * (w.d // 16), w.d), scale / np.sqrt(w.d))
 
 
 def selector_tables(w: Workload, scale: float = 1.0):

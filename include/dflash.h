@@ -71,6 +71,26 @@ int dflash_conv2tap(const dflash_bf16* x, const dflash_bf16* prev, const dflash_
                     const dflash_bf16* a1, dflash_bf16* y, int B, int P, int d, void* stream);
 
 /*
+ * Two-tap conv with content-dependent taps.
+ * "DFlash 2: Keep Drafting Parallel", section "a lightweight local
+ * convolution": each coefficient is a learnable base kernel plus a small
+ * correction computed from the current hidden state, one correction shared
+ * by every 16 channels.  With G = d / 16 and the correction projection
+ * Wc [2G, d] (rows 0..G-1: tap 0, rows G..2G-1: tap 1):
+ *   delta_j[b,t,g] = sum_c x[b,t,c] * Wc[j*G + g, c]
+ *   y[b,t,c] = (a0[c] + delta_0[b,t,c/16]) * x[b,t,c]
+ *            + (a1[c] + delta_1[b,t,c/16]) * x[b,t-1,c],  x[b,-1,:] = prev[b,:]
+ * x [B,P,d], prev [B,d] (NULL: zeros), a0, a1 [d], Wc [2G,d], y [B,P,d]: bf16.
+ * ws: device workspace of dflash_conv2tap_dynamic_workspace(B,P,d) bytes
+ * (holds delta in fp32).  d % 16 == 0, d >= 128; all pointers 16-byte
+ * aligned.  Runs the tensor-core GEMM for delta, then a streaming kernel.
+ */
+size_t dflash_conv2tap_dynamic_workspace(int B, int P, int d);
+int dflash_conv2tap_dynamic(const dflash_bf16* x, const dflash_bf16* prev, const dflash_bf16* a0,
+                            const dflash_bf16* a1, const dflash_bf16* wc, dflash_bf16* y, int B, int P, int d,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Bytes of device workspace dflash_lmhead_topk needs for these sizes
  * (0 when the sizes are invalid).
  */
@@ -133,6 +153,18 @@ int dflash_lmhead_topk_static(const dflash_bf16* H, const dflash_bf16* W, int M,
  */
 int dflash_lmhead_logits_debug(const dflash_bf16* H, const dflash_bf16* W, int M, int V, int d,
                                float* z, void* ws, size_t ws_bytes, int* dev_status, void* stream);
+
+/*
+ * Plain bf16 GEMM on the LM head's tensor-core path:
+ *   C[m,n] = sum_k A[m,k] * B[n,k]      (fp32 accumulation, fp32 out)
+ * A [M, K] bf16, B [N, K] bf16 (both K-major, 16-byte aligned), C [M, N] fp32
+ * row-major (16-byte aligned).  K % 8 == 0, N >= 16.  Needs no workspace.
+ * It computes the projections of the dynamic conv's tap corrections and of
+ * the context-gated pair scorer ("DFlash 2: Keep Drafting Parallel",
+ * sections "a lightweight local convolution" and "a lightweight path
+ * selector").
+ */
+int dflash_gemm_bf16(const dflash_bf16* A, const dflash_bf16* B, float* C, int M, int N, int K, void* stream);
 
 /*
  * Path selection over the candidate lists.

@@ -16,6 +16,9 @@ no blocking, fusion or reordering beyond what each definition states.
 
 Pins (``tests/test_oracle_*.py``, run with ``-m "not gpu"``):
   conv2tap      hand-worked case, identity/shift taps, marker inputs
+  conv2tap_dynamic
+                zero correction = the static conv, a hand-worked case, a
+                correction confined to its 16-channel group
   lmhead_topk   exact rational/decimal brute force on tiny shapes, heap
                 selection, the uniform-logit case (lse = log V)
   argmax_tokens exact brute force, tie to the lowest index
@@ -24,10 +27,10 @@ Pins (``tests/test_oracle_*.py``, run with ``-m "not gpu"``):
                 pair table, the E = 0 case (= the top-1 path), a hand case
   verify        hand cases and the Table 1 closed form (4.27 / 6.79)
 """
-from .conv import conv2tap
+from .conv import conv2tap, conv2tap_dynamic
 from .lmhead import logits, lmhead_topk, argmax_tokens, topk_margin_ok
 from .selector import pair_scores, viterbi, viterbi_two_best, path_select
 from .verify import verify
 
-__all__ = ["conv2tap", "logits", "lmhead_topk", "argmax_tokens", "topk_margin_ok",
+__all__ = ["conv2tap", "conv2tap_dynamic", "logits", "lmhead_topk", "argmax_tokens", "topk_margin_ok",
            "pair_scores", "viterbi", "viterbi_two_best", "path_select", "verify"]

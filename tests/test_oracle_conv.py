@@ -48,3 +48,55 @@ def test_single_position_block():
     y = oracle.conv2tap(_bits(x), _bits(prev), _bits([1.0, 0.5]), _bits([0.25, 0.125]))
     np.testing.assert_array_equal(y, [[[2.0 + 1.0, -0.5 + 1.0]]])
 
+
+
+def _dyn_hand(golden):
+    g = golden("conv_dynamic_hand.json")
+    d = 16
+    x = np.zeros((1, 2, d), np.float32)
+    x[0, 0, :4] = g["x_t0"]
+    x[0, 1, :4] = g["x_t1"]
+    prev = np.zeros((1, d), np.float32)
+    prev[0, :4] = g["prev"]
+    a0 = np.zeros(d, np.float32); a0[:4] = g["a0"]
+    a1 = np.zeros(d, np.float32); a1[:4] = g["a1"]
+    wc = np.zeros((2, d), np.float32)
+    wc[0, 0] = 0.5
+    wc[1, 1] = 0.25
+    return g, x, prev, a0, a1, wc
+
+
+def test_dynamic_hand_worked(golden):
+    g, x, prev, a0, a1, wc = _dyn_hand(golden)
+    y = oracle.conv2tap_dynamic(_bits(x), _bits(prev), _bits(a0), _bits(a1), _bits(wc))
+    np.testing.assert_array_equal(y[0, 0, :4], g["y_t0"])
+    np.testing.assert_array_equal(y[0, 1, :4], g["y_t1"])
+
+
+def test_dynamic_zero_correction_is_static_conv():
+    from block_draft_synth import workload, conv_input, conv_taps
+    w = workload(0)
+    x, prev = conv_input(w)
+    a0, a1 = conv_taps(w)
+    wc = np.zeros((2 * w.d // 16, w.d), np.uint16)
+    np.testing.assert_array_equal(oracle.conv2tap_dynamic(x, prev, a0, a1, wc),
+                                  oracle.conv2tap(x, prev, a0, a1))
+
+
+def test_dynamic_correction_stays_in_its_group():
+    """A correction row for group g changes channels 16g..16g+15 only (catches
+    a wrong group index or a missing broadcast)."""
+    from block_draft_synth import workload, conv_input, conv_taps
+    w = workload(0)
+    x, prev = conv_input(w)
+    a0, a1 = conv_taps(w)
+    G = w.d // 16
+    base = oracle.conv2tap(x, prev, a0, a1)
+    for j, g in ((0, 3), (1, 7)):
+        wc = np.zeros((2 * G, w.d), np.float32)
+        wc[j * G + g, :] = 0.01
+        y = oracle.conv2tap_dynamic(x, prev, a0, a1, _bits(wc))
+        changed = np.abs(y - base).max(axis=(0, 1)) > 0
+        assert changed[16 * g:16 * g + 16].all()
+        changed[16 * g:16 * g + 16] = False
+        assert not changed.any()

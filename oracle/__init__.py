@@ -26,11 +26,23 @@ Pins (``tests/test_oracle_*.py``, run with ``-m "not gpu"``):
                 exhaustive 16^L enumeration for L <= 4 on an exact rational
                 pair table, the E = 0 case (= the top-1 path), a hand case
   verify        hand cases and the Table 1 closed form (4.27 / 6.79)
+  greedy_walk / sample_walk
+                a hand case where greedy misses the anchored max-sum path,
+                exact rational scores on random tiny cases, the T -> 0 limit
+                (= greedy), the E = 0 closed form at T = 1 (the renormalised
+                top-16), and the path distribution integrated over a grid of
+                uniforms against exact conditional softmaxes
+  verify_rejection
+                hand cases, and the output-distribution theorem: the first
+                emitted token is distributed exactly as the target's p_0
+                (integrated over grids of both uniforms)
 """
 from .conv import conv2tap, conv2tap_dynamic
 from .lmhead import logits, lmhead_topk, argmax_tokens, topk_margin_ok
 from .selector import pair_scores, viterbi, viterbi_two_best, path_select
 from .verify import verify
+from .walks import anchor_scores, greedy_walk, sample_walk, verify_rejection, inverse_cdf
 
 __all__ = ["conv2tap", "conv2tap_dynamic", "logits", "lmhead_topk", "argmax_tokens", "topk_margin_ok",
-           "pair_scores", "viterbi", "viterbi_two_best", "path_select", "verify"]
+           "pair_scores", "viterbi", "viterbi_two_best", "path_select", "verify",
+           "anchor_scores", "greedy_walk", "sample_walk", "verify_rejection", "inverse_cdf"]

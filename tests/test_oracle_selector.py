@@ -11,18 +11,9 @@ import pytest
 
 import oracle
 from block_draft_synth import f32_to_bf16_bits, synthetic_topk, rng_for
+from exact import exact_pairs
 
 K = 16
-
-
-def _bf(b):
-    b = int(b)
-    sign = -1 if b & 0x8000 else 1
-    exp = (b >> 7) & 0xFF
-    man = b & 0x7F
-    if exp == 0:
-        return sign * Fraction(man, 1 << 133)
-    return sign * Fraction(128 + man, 128) * Fraction(2) ** (exp - 127)
 
 
 def _tables(seed, V, r, scale):
@@ -32,27 +23,7 @@ def _tables(seed, V, r, scale):
     return E, M
 
 
-def _exact_pairs(logp, idx, E, M, b, L):
-    r = M.shape[0]
-    Mf = [[_bf(M[s, t]) for t in range(r)] for s in range(r)]
-    rows = {}
-    for i in range(L):
-        for j in range(K):
-            c = int(idx[b * L + i, j])
-            if c not in rows:
-                rows[c] = [_bf(E[c, s]) for s in range(r)]
-    lp = [[Fraction(float(logp[b * L + i, j])) for j in range(K)] for i in range(L)]
-    S = []
-    for i in range(L - 1):
-        Si = [[None] * K for _ in range(K)]
-        for j in range(K):
-            ea = rows[int(idx[b * L + i, j])]
-            u = [sum(ea[s] * Mf[s][t] for s in range(r)) for t in range(r)]
-            for k in range(K):
-                eb = rows[int(idx[b * L + i + 1, k])]
-                Si[j][k] = lp[i][j] + lp[i + 1][k] + sum(u[t] * eb[t] for t in range(r))
-        S.append(Si)
-    return S
+_exact_pairs = exact_pairs
 
 
 def _brute(S, L):

@@ -19,10 +19,13 @@ from ._binding import (  # noqa: F401
     dflash_lmhead_topk,
     dflash_lmhead_topk_workspace,
     dflash_path_select,
+    dflash_path_walk,
     dflash_select_verify,
     dflash_lmhead_topk_static,
     dflash_status_string,
     dflash_verify,
+    dflash_verify_rejection,
+    dflash_verify_rejection_workspace,
     lib,
     workspace,
 )

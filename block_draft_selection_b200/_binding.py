@@ -52,6 +52,11 @@ def _load():
         "dflash_gemm_bf16": (i32, [vp, vp, vp, i32, i32, i32, vp]),
         "dflash_conv2tap_dynamic_workspace": (sz, [i32, i32, i32]),
         "dflash_conv2tap_dynamic": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, sz, vp]),
+        "dflash_path_walk": (i32, [vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, i32, i32, i32, i32,
+                                   vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "dflash_verify_rejection_workspace": (sz, [i32, i32, i32]),
+        "dflash_verify_rejection": (i32, [vp, ctypes.c_float, vp, vp, vp, vp, vp, vp, i32, i32, i32,
+                                          vp, vp, vp, sz, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -268,4 +273,71 @@ def dflash_verify(draft, target, accept_len=None, next_token=None, stream=None):
     next_token = _out(next_token, "next_token", torch.int32, (B,), draft.device)
     _check("dflash_verify", lib.dflash_verify(_ptr(draft), _ptr(target), B, L, _ptr(accept_len),
                                               _ptr(next_token), _stream(stream)))
+    return accept_len, next_token
+
+
+def dflash_path_walk(topk_logp, topk_idx, E, Msel, anchor, B, L, uniforms=None, temperature=1.0,
+                     path_tok=None, path_slot=None, path_score=None, path_q=None, want_q=True,
+                     target=None, accept_len=None, next_token=None, dev_status=None, stream=None):
+    """Walk from the last verified token: greedy when `uniforms` is None, else sampled
+    at `temperature`.  Returns (path_tok, path_slot, path_score, path_q or None,
+    accept_len or None, next_token or None); the last two only when `target` is given."""
+    _need(topk_logp, "topk_logp", torch.float32, (B * L, K_TOP))
+    _need(topk_idx, "topk_idx", torch.int32, (B * L, K_TOP))
+    _need(E, "E", torch.bfloat16)
+    V, r = E.shape
+    _need(Msel, "Msel", torch.bfloat16, (r, r))
+    _need(anchor, "anchor", torch.int32, (B,))
+    dev = topk_logp.device
+    if uniforms is not None:
+        _need(uniforms, "uniforms", torch.float32, (B, L))
+    path_tok = _out(path_tok, "path_tok", torch.int32, (B, L), dev)
+    path_slot = _out(path_slot, "path_slot", torch.int32, (B, L), dev)
+    path_score = _out(path_score, "path_score", torch.float32, (B,), dev)
+    if uniforms is not None and (want_q or path_q is not None):
+        path_q = _out(path_q, "path_q", torch.float32, (B, L, K_TOP), dev)
+    else:
+        path_q = None
+    if target is not None:
+        _need(target, "target", torch.int32, (B, L + 1))
+        accept_len = _out(accept_len, "accept_len", torch.int32, (B,), dev)
+        next_token = _out(next_token, "next_token", torch.int32, (B,), dev)
+    else:
+        accept_len = next_token = None
+    _check("dflash_path_walk", lib.dflash_path_walk(
+        _ptr(topk_logp), _ptr(topk_idx), _ptr(E), _ptr(Msel), _ptr(anchor), _ptr(uniforms),
+        float(temperature), B, L, K_TOP, r, V, _ptr(path_tok), _ptr(path_slot), _ptr(path_score),
+        _ptr(path_q), _ptr(target), _ptr(accept_len), _ptr(next_token), _ptr(dev_status), _stream(stream)))
+    return path_tok, path_slot, path_score, path_q, accept_len, next_token
+
+
+def dflash_verify_rejection_workspace(B: int, L: int, V: int) -> int:
+    return int(lib.dflash_verify_rejection_workspace(B, L, V))
+
+
+def dflash_verify_rejection(target_logits, temperature, draft, draft_slot, cand_idx, draft_q, u_accept,
+                            u_resample, accept_len=None, next_token=None, ws=None, dev_status=None,
+                            stream=None):
+    """Rejection-sampling verification.  target_logits [B*(L+1), V] f32; draft, draft_slot
+    [B, L] i32; cand_idx [B*L, 16] i32; draft_q [B, L, 16] f32; u_accept [B, L] f32;
+    u_resample [B] f32.  Returns (accept_len [B] i32, next_token [B] i32)."""
+    _need(draft, "draft", torch.int32)
+    B, L = draft.shape
+    _need(target_logits, "target_logits", torch.float32)
+    V = target_logits.shape[1]
+    _need(target_logits, "target_logits", torch.float32, (B * (L + 1), V))
+    _need(draft_slot, "draft_slot", torch.int32, (B, L))
+    _need(cand_idx, "cand_idx", torch.int32, (B * L, K_TOP))
+    _need(draft_q, "draft_q", torch.float32, (B, L, K_TOP))
+    _need(u_accept, "u_accept", torch.float32, (B, L))
+    _need(u_resample, "u_resample", torch.float32, (B,))
+    dev = draft.device
+    accept_len = _out(accept_len, "accept_len", torch.int32, (B,), dev)
+    next_token = _out(next_token, "next_token", torch.int32, (B,), dev)
+    if ws is None:
+        ws = torch.empty(max(1, dflash_verify_rejection_workspace(B, L, V)), dtype=torch.uint8, device=dev)
+    _check("dflash_verify_rejection", lib.dflash_verify_rejection(
+        _ptr(target_logits), float(temperature), _ptr(draft), _ptr(draft_slot), _ptr(cand_idx),
+        _ptr(draft_q), _ptr(u_accept), _ptr(u_resample), B, L, V, _ptr(accept_len), _ptr(next_token),
+        _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream)))
     return accept_len, next_token

@@ -31,7 +31,8 @@
 //          vocabulary-strided (W shared through L2 across concurrent token
 //          tiles) or long runs of one token tile over a vocabulary range.
 // No load uses cluster multicast: every CTA fetches its own tiles.
-// Kernel 2 (merge_kernel) folds a row's partials: one warp per row.
+// Kernel 2 (merge_kernel_rank) merges a row's partial records: one CTA per
+// row picks the top-16 by a threshold and a parallel rank count.
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -599,77 +600,172 @@ __device__ __forceinline__ void fold_records(TopState& st, const Partial* base, 
   }
 }
 
-// Few records per row: one warp per row.
-__global__ void __launch_bounds__(128) merge_kernel(const Partial* __restrict__ part, int M, int P,
-                                                    float* __restrict__ topk_logp,
-                                                    int32_t* __restrict__ topk_idx,
-                                                    float* __restrict__ lse) {
-  const int lane = threadIdx.x & 31;
-  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  pdl_wait();
-  pdl_trigger();
-  if (row >= M) return;
-  TopState st;
-  st.reset();
-  fold_records(st, part + static_cast<size_t>(row) * P, lane, 32, P);
-  float v;
-  int ix;
-  warp_merge(st, v, ix);
-  // one lane's lse for every slot: the butterfly leaves lanes' (m, s) equal
-  // only up to rounding, which could reorder log-probs of near-equal logits
-  const float row_lse = __shfl_sync(0xffffffffu, st.m + logf(st.s), 0);
-  if (lane < KTOP) {
-    topk_logp[static_cast<size_t>(row) * KTOP + lane] = v - row_lse;
-    topk_idx[static_cast<size_t>(row) * KTOP + lane] = ix;
-  }
-  if (lane == 0 && lse != nullptr) lse[row] = row_lse;
-}
+// Threshold-and-rank merge: one CTA per row, no serial list merging.
+// Every record is a sorted list, so any 16 entries of the row bound its 16th
+// best value from below.  Pass 1 merges the records' (m, s) and takes as that
+// bound tau the 16th largest of the records' leading entries (the first J of
+// each record, J = ceil(16 / P), so that there are at least 16 of them),
+// found by counting for each leading entry how many are at least as large;
+// tau is raised to the largest 16th entry of any one record if that is
+// higher.  Pass 2 gathers every entry >= tau (a prefix of each record) into
+// shared memory -- typically a few more than 16.  Pass 3 gives each gathered
+// entry its rank under the full order (value descending, index ascending)
+// by counting the entries ahead of it; the entries ranked 0..15 are the
+// row's top-16.  Ranks are distinct because a vocabulary index appears in
+// exactly one record.  If ties overflow the shared buffers, the CTA falls
+// back to folding the records list by list.
+constexpr int MR_CAP = 1024;
 
-// Many records per row: one CTA of 256 threads per row; eight warp lists are
-// merged again by warp 0.
-__global__ void __launch_bounds__(256) merge_kernel_wide(const Partial* __restrict__ part, int M, int P,
-                                                         float* __restrict__ topk_logp,
-                                                         int32_t* __restrict__ topk_idx,
-                                                         float* __restrict__ lse) {
-  __shared__ float sv[8][KTOP];
-  __shared__ int si[8][KTOP];
-  __shared__ float sm[8], ss[8];
-  const int lane = threadIdx.x & 31;
-  const int w = threadIdx.x >> 5;
+template <int NT>
+__global__ void __launch_bounds__(NT) merge_kernel_rank(const Partial* __restrict__ part, int M, int P,
+                                                        float* __restrict__ topk_logp,
+                                                        int32_t* __restrict__ topk_idx,
+                                                        float* __restrict__ lse) {
+  constexpr int NW = NT / 32;
+  __shared__ float cv[MR_CAP];
+  __shared__ int ci[MR_CAP];
+  __shared__ float red_m[NW], red_s[NW], red_t[NW];
+  __shared__ float fv[NW][KTOP];
+  __shared__ int fi[NW][KTOP];
+  __shared__ int count, nhead;
+  __shared__ float sh_lse, sh_tau;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int row = blockIdx.x;
+  const Partial* base = part + static_cast<size_t>(row) * P;
   pdl_wait();
   pdl_trigger();
-  TopState st;
-  st.reset();
-  fold_records(st, part + static_cast<size_t>(row) * P, threadIdx.x, blockDim.x, P);
-  float v;
-  int ix;
-  warp_merge(st, v, ix);
-  if (lane < KTOP) {
-    sv[w][lane] = v;
-    si[w][lane] = ix;
-  }
-  if (lane == 0) {
-    sm[w] = st.m;
-    ss[w] = st.s;
+  if (tid == 0) {
+    count = 0;
+    nhead = 0;
   }
   __syncthreads();
-  if (w != 0) return;
-  TopState fin;
-  fin.reset();
-  if (lane < 8) fin.merge_lse(sm[lane], ss[lane]);
+  const int J = P >= KTOP ? 1 : (KTOP + P - 1) / P;  // leading entries per record
+
+  // pass 1: (m, s) of the row, the largest 16th entry, the leading entries
+  TopState st;  // only m and s are used
+  st.m = -INFINITY;
+  st.s = 0.f;
+  float tau16 = -INFINITY;
+  for (int q = tid; q < P; q += NT) {
+    const float* r = reinterpret_cast<const float*>(base + q);
+    const float4 h = __ldg(reinterpret_cast<const float4*>(r));
+    st.merge_lse(h.x, h.y);
+    tau16 = fmaxf(tau16, __ldg(r + 4 + (KTOP - 1)));
+    const int pos = atomicAdd(&nhead, J);
+    for (int j = 0; j < J; ++j)
+      if (pos + j < MR_CAP) cv[pos + j] = __ldg(r + 4 + j);
+  }
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int c = q * 32 + lane;  // candidate c of the 8 x 16 warp lists
-    fin.insert(sv[c >> 4][c & 15], si[c >> 4][c & 15]);
+  for (int off = 16; off; off >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, st.m, off);
+    const float s2 = __shfl_xor_sync(0xffffffffu, st.s, off);
+    st.merge_lse(m2, s2);
+    tau16 = fmaxf(tau16, __shfl_xor_sync(0xffffffffu, tau16, off));
   }
-  warp_merge(fin, v, ix);
-  const float row_lse = __shfl_sync(0xffffffffu, fin.m + logf(fin.s), 0);
-  if (lane < KTOP) {
-    topk_logp[static_cast<size_t>(row) * KTOP + lane] = v - row_lse;
-    topk_idx[static_cast<size_t>(row) * KTOP + lane] = ix;
+  if (lane == 0) {
+    red_m[w] = st.m;
+    red_s[w] = st.s;
   }
-  if (lane == 0 && lse != nullptr) lse[row] = row_lse;
+  __syncthreads();
+  // the 16th largest leading entry: the largest h with #{h' >= h} >= 16
+  const int nh = nhead < MR_CAP ? nhead : MR_CAP;
+  float th = -INFINITY;
+  for (int c = tid; c < nh; c += NT) {
+    const float h = cv[c];
+    int ge = 0;
+    for (int j = 0; j < nh; ++j) ge += cv[j] >= h ? 1 : 0;
+    if (ge >= KTOP) th = fmaxf(th, h);
+  }
+  th = fmaxf(th, tau16);
+#pragma unroll
+  for (int off = 16; off; off >>= 1) th = fmaxf(th, __shfl_xor_sync(0xffffffffu, th, off));
+  if (lane == 0) red_t[w] = th;
+  __syncthreads();
+  if (tid == 0) {
+    float t = red_t[0];
+    for (int k = 1; k < NW; ++k) {
+      st.merge_lse(red_m[k], red_s[k]);
+      t = fmaxf(t, red_t[k]);
+    }
+    sh_lse = st.m + logf(st.s);
+    sh_tau = t;
+  }
+  __syncthreads();  // also: every read of the leading entries is done
+  const float tau = sh_tau;
+  const float row_lse = sh_lse;
+
+  // pass 2: gather the entries >= tau (a prefix of each record)
+  for (int q = tid; q < P; q += NT) {
+    const float4* r = reinterpret_cast<const float4*>(base + q);
+    float v[KTOP];
+    int ix[KTOP];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float4 a = __ldg(r + 1 + k);
+      const float4 b = __ldg(r + 5 + k);
+      v[4 * k] = a.x, v[4 * k + 1] = a.y, v[4 * k + 2] = a.z, v[4 * k + 3] = a.w;
+      ix[4 * k] = __float_as_int(b.x), ix[4 * k + 1] = __float_as_int(b.y);
+      ix[4 * k + 2] = __float_as_int(b.z), ix[4 * k + 3] = __float_as_int(b.w);
+    }
+    int c = 0;
+#pragma unroll
+    for (int k = 0; k < KTOP; ++k) c += (v[k] >= tau && ix[k] != 0x7fffffff) ? 1 : 0;
+    if (c) {
+      const int pos = atomicAdd(&count, c);
+#pragma unroll
+      for (int k = 0; k < KTOP; ++k) {
+        if (k < c && pos + k < MR_CAP) {
+          cv[pos + k] = v[k];
+          ci[pos + k] = ix[k];
+        }
+      }
+    }
+  }
+  __syncthreads();
+  const int n = count;
+  float* out_v = topk_logp + static_cast<size_t>(row) * KTOP;
+  int32_t* out_i = topk_idx + static_cast<size_t>(row) * KTOP;
+  if (n <= MR_CAP) {
+    // pass 3: rank of each gathered entry
+    for (int c = tid; c < n; c += NT) {
+      const float v = cv[c];
+      const int ix = ci[c];
+      int rank = 0;
+      for (int j = 0; j < n; ++j) rank += better(cv[j], ci[j], v, ix) ? 1 : 0;
+      if (rank < KTOP) {
+        out_v[rank] = v - row_lse;
+        out_i[rank] = ix;
+      }
+    }
+    if (tid >= n && tid < KTOP) {  // fewer than 16 entries in the whole row
+      out_v[tid] = -INFINITY;
+      out_i[tid] = 0x7fffffff;
+    }
+  } else {
+    // ties overflowed a buffer: fold the records list by list
+    TopState fs;
+    fs.reset();
+    fold_records(fs, base, tid, NT, P);
+    float v;
+    int ix;
+    warp_merge(fs, v, ix);
+    if (lane < KTOP) {
+      fv[w][lane] = v;
+      fi[w][lane] = ix;
+    }
+    __syncthreads();
+    if (w == 0) {
+      TopState fin;
+      fin.reset();
+      for (int c = lane; c < NW * KTOP; c += 32) fin.insert(fv[c / KTOP][c % KTOP], fi[c / KTOP][c % KTOP]);
+      warp_merge(fin, v, ix);
+      if (lane < KTOP) {
+        out_v[lane] = v - row_lse;
+        out_i[lane] = ix;
+      }
+    }
+  }
+  if (tid == 0 && lse != nullptr) lse[row] = row_lse;
 }
 
 // ------------------------------------------------------------ host side ----
@@ -929,12 +1025,10 @@ static int launch(const dflash_bf16* H, const dflash_bf16* W, int M, int V, int 
   if (z_dbg == nullptr && !store_only) {
     const Partial* part = p.part;
     cudaError_t me;
-    if (p.P >= 64) {
-      me = launch_kernel(merge_kernel_wide, dim3(M), dim3(256), 0, st, part, M, p.P, topk_logp, topk_idx, lse);
+    if (p.P > 128) {
+      me = launch_kernel(merge_kernel_rank<256>, dim3(M), dim3(256), 0, st, part, M, p.P, topk_logp, topk_idx, lse);
     } else {
-      const int rows_per_cta = 4;
-      me = launch_kernel(merge_kernel, dim3((M + rows_per_cta - 1) / rows_per_cta), dim3(32 * rows_per_cta), 0, st,
-                         part, M, p.P, topk_logp, topk_idx, lse);
+      me = launch_kernel(merge_kernel_rank<128>, dim3(M), dim3(128), 0, st, part, M, p.P, topk_logp, topk_idx, lse);
     }
     if (me != cudaSuccess) return DFLASH_ERR_CUDA;
   }

@@ -22,6 +22,14 @@
 //      (h,k) takes the max over j in half h of delta[j] + S[j,k], one xor-16
 //      shuffle joins the halves, backpointers go to shared memory; then a
 //      16-lane argmax, a backtrack and (optionally) greedy verification.
+//
+// The same kernel also walks from the last verified ("anchor") token, the
+// walk the section describes: greedily following the best successor, or
+// drawing each successor from softmax(score / T) over the 16 candidates.
+// For these walks an extra internal position 0 holds the anchor (16 copies
+// of its E row, log-probability 0), so the first pair table is
+//   S_a[k] = lp[0,k] + (e_anchor M) . e_{c_0k}
+// and internal position p >= 1 is drafted position p - 1.
 #include <mutex>
 
 #include <cooperative_groups.h>
@@ -76,13 +84,102 @@ __host__ __device__ inline Layout layout(int L, int r) {
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+enum Walk { WALK_VITERBI = 0, WALK_GREEDY = 1, WALK_SAMPLE = 2 };
+
+struct WalkArgs {
+  const int32_t* anchor;   // [B] last verified token (greedy / sample)
+  const float* uniforms;   // [B, L] one uniform per drafted position (sample)
+  float inv_t;             // 1 / temperature (sample)
+  float* path_q;           // [B, L, 16] distribution each slot was drawn from (nullable)
+};
+
+// One warp walks L steps from the anchor over the pair tables in shared
+// memory (table i: row = previous slot, column = next slot).  Lane (h, k)
+// holds column k; both half-warps compute the same values.
+//   greedy: next = argmax_k S_i[cur, k] (ties: lowest k)
+//   sample: q = softmax(S_i[cur, :] / T); next = the smallest k whose
+//           cumulative q exceeds u_i (inverse CDF in slot order)
+template <int WALK>
+__device__ __forceinline__ void walk_from_anchor(const float* Ss, const int* toks, int L, int b, const WalkArgs& wa,
+                                                 int32_t* path_tok, int32_t* path_slot, float* path_score,
+                                                 const int32_t* target, int32_t* accept_len, int32_t* next_token) {
+  const int lane = threadIdx.x & 31;
+  const int k = lane & 15;
+  const size_t row0 = static_cast<size_t>(b) * L;
+  // the uniforms of this block, one per lane (read before the serial walk)
+  float u_mine = 0.f;
+  if (WALK == WALK_SAMPLE && lane < L) u_mine = __ldg(wa.uniforms + row0 + lane);
+  int cur = 0;
+  int my_slot = 0;  // lane i keeps the slot chosen at position i
+  float score = 0.f;
+  for (int i = 0; i < L; ++i) {
+    const float v = Ss[(i * KC + cur) * KC + k];
+    int nk;
+    if (WALK == WALK_GREEDY) {
+      float bv = v;
+      int bk = k;
+#pragma unroll
+      for (int off = 1; off < 16; off <<= 1) {
+        const float v2 = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int k2 = __shfl_xor_sync(0xffffffffu, bk, off);
+        if (v2 > bv || (v2 == bv && k2 < bk)) {
+          bv = v2;
+          bk = k2;
+        }
+      }
+      nk = bk;
+    } else {
+      float m = v;
+#pragma unroll
+      for (int off = 1; off < 16; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      const float e = expf((v - m) * wa.inv_t);
+      // inclusive prefix sum over the 16 lanes of each half
+      float c = e;
+#pragma unroll
+      for (int off = 1; off < 16; off <<= 1) {
+        const float t = __shfl_up_sync(0xffffffffu, c, off, 16);
+        if (k >= off) c += t;
+      }
+      const float total = __shfl_sync(0xffffffffu, c, 15);
+      const float u = __shfl_sync(0xffffffffu, u_mine, i);
+      const unsigned over = __ballot_sync(0xffffffffu, c > u * total) & 0xffffu;
+      nk = over ? __ffs(over) - 1 : 15;
+      if (wa.path_q && lane < 16) wa.path_q[(row0 + i) * KC + k] = e / total;
+    }
+    score += __shfl_sync(0xffffffffu, v, nk);
+    if (lane == i) my_slot = nk;
+    cur = nk;
+  }
+  const bool in_block = lane < L;
+  const int my_tok = in_block ? toks[(lane + 1) * KC + my_slot] : 0;
+  if (in_block) {
+    path_tok[row0 + lane] = my_tok;
+    if (path_slot) path_slot[row0 + lane] = my_slot;
+  }
+  if (path_score && lane == 0) path_score[b] = score;
+  if (target != nullptr) {
+    const int32_t* tg = target + static_cast<size_t>(b) * (L + 1);
+    const bool differs = in_block && my_tok != __ldg(tg + lane);
+    const unsigned mask = __ballot_sync(0xffffffffu, differs);
+    const int n = mask ? __ffs(mask) - 1 : L;
+    if (lane == 0) {
+      accept_len[b] = n + 1;
+      next_token[b] = __ldg(tg + n);
+    }
+  }
+}
+
+template <int WALK>
 __global__ void __launch_bounds__(THREADS) path_select_kernel(
     const float* __restrict__ topk_logp, const int32_t* __restrict__ topk_idx, const uint16_t* __restrict__ E,
     const uint16_t* __restrict__ Msel, int L, int r, int V, int32_t* __restrict__ path_tok,
     int32_t* __restrict__ path_slot, float* __restrict__ path_score, float* __restrict__ pair_dbg, int* status,
-    const int32_t* __restrict__ target, int32_t* __restrict__ accept_len, int32_t* __restrict__ next_token, int Q) {
+    const int32_t* __restrict__ target, int32_t* __restrict__ accept_len, int32_t* __restrict__ next_token, int Q,
+    WalkArgs wa) {
   extern __shared__ __align__(16) uint8_t smem[];
-  const Layout lo = layout(L, r);
+  constexpr int OFF = WALK == WALK_VITERBI ? 0 : 1;  // internal positions before drafted position 0
+  const int Li = L + OFF;                            // internal positions
+  const Layout lo = layout(Li, r);
   uint16_t* Ms = reinterpret_cast<uint16_t*>(smem + lo.m_off);
   uint16_t* Es = reinterpret_cast<uint16_t*>(smem + lo.e_off);
   float* Us = reinterpret_cast<float*>(smem + lo.u_off);
@@ -99,7 +196,7 @@ __global__ void __launch_bounds__(THREADS) path_select_kernel(
   const int nthr = blockDim.x;
   const int r8 = r / 8;
   const size_t row0 = static_cast<size_t>(b) * L;
-  const int npos = L - 1;
+  const int npos = Li - 1;  // pair tables
   // Scores go to the leader's shared memory (this CTA's own when Q == 1).
   // The leader's shared memory may be written only once every CTA of the
   // cluster runs: arrive now, wait just before the first remote store.
@@ -120,9 +217,22 @@ __global__ void __launch_bounds__(THREADS) path_select_kernel(
   // One pass: every load here depends only on global inputs, so the index
   // reads, the E-row gathers that follow them and the copy of M are all in
   // flight together.
-  for (int q = tid; q < L * KC; q += nthr) {
-    lps[q] = __ldg(topk_logp + row0 * KC + q);
-    int c = __ldg(topk_idx + row0 * KC + q);
+  int anchor_tok = 0;
+  if (OFF) {
+    anchor_tok = __ldg(wa.anchor + b);
+    if (anchor_tok < 0 || anchor_tok >= V) {
+      if (tid == 0) set_status(status, DFLASH_ERR_BAD_INDEX);
+      anchor_tok = 0;
+    }
+  }
+  for (int q = tid; q < Li * KC; q += nthr) {
+    if (OFF && q < KC) {  // the anchor: 16 copies, no unary term
+      lps[q] = 0.f;
+      toks[q] = anchor_tok;
+      continue;
+    }
+    lps[q] = __ldg(topk_logp + row0 * KC + (q - OFF * KC));
+    int c = __ldg(topk_idx + row0 * KC + (q - OFF * KC));
     if (c < 0 || c >= V) {
       set_status(status, DFLASH_ERR_BAD_INDEX);
       c = 0;
@@ -134,11 +244,11 @@ __global__ void __launch_bounds__(THREADS) path_select_kernel(
     uint4* Mv = reinterpret_cast<uint4*>(Ms);
     for (int q = tid; q < r * r8; q += nthr) Mv[q] = __ldg(Mg + q);
   }
-  for (int q = tid; q < L * KC * r8; q += nthr) {
+  for (int q = tid; q < Li * KC * r8; q += nthr) {
     const int cand = q / r8;
     const int v8 = q - cand * r8;
     if (!needs_pos(cand / KC)) continue;
-    int c = __ldg(topk_idx + row0 * KC + cand);
+    int c = (OFF && cand < KC) ? anchor_tok : __ldg(topk_idx + row0 * KC + (cand - OFF * KC));
     c = (c < 0 || c >= V) ? 0 : c;
     const uint4 val = __ldg(reinterpret_cast<const uint4*>(E + static_cast<size_t>(c) * r) + v8);
     *reinterpret_cast<uint4*>(Es + static_cast<size_t>(cand) * lo.rp + v8 * 8) = val;
@@ -203,7 +313,7 @@ __global__ void __launch_bounds__(THREADS) path_select_kernel(
       }
       const float sc = (lps[i * KC + j] + lps[(i + 1) * KC + k]) + acc;
       S_out[(i * KC + j) * KC + k] = sc;
-      if (pair_dbg) pair_dbg[((static_cast<size_t>(b) * npos + i) * KC + j) * KC + k] = sc;
+      if (WALK == WALK_VITERBI && pair_dbg) pair_dbg[((static_cast<size_t>(b) * npos + i) * KC + j) * KC + k] = sc;
     }
     __syncthreads();
   }
@@ -212,6 +322,11 @@ __global__ void __launch_bounds__(THREADS) path_select_kernel(
   if (Q > 1) {
     cooperative_groups::this_cluster().sync();  // every CTA's scores have landed
     if (q_rank != 0) return;
+  }
+  if (WALK != WALK_VITERBI) {
+    if (tid < 32) walk_from_anchor<WALK>(Ss, toks, L, b, wa, path_tok, path_slot, path_score, target, accept_len,
+                                         next_token);
+    return;
   }
   if (tid < 32) {
     const int lane = tid;
@@ -293,19 +408,23 @@ __global__ void __launch_bounds__(THREADS) path_select_kernel(
 namespace dflash {
 namespace sel {
 
+template <int WALK>
 static int launch(const float* topk_logp, const int32_t* topk_idx, const dflash_bf16* E, const dflash_bf16* Msel,
                   int B, int L, int K, int r, int V, int32_t* path_tok, int32_t* path_slot, float* path_score,
                   float* pair_scores_dbg, const int32_t* target, int32_t* accept_len, int32_t* next_token,
-                  int* dev_status, void* stream) {
+                  int* dev_status, void* stream, WalkArgs wa) {
   if (!topk_logp || !topk_idx || !E || !Msel || !path_tok) return DFLASH_ERR_INVALID_ARG;
   if (K != KC || B < 1 || L < 1 || L > 16 || r < 8 || r > 128 || r % 8 != 0 || V < 1)
     return DFLASH_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(E) | reinterpret_cast<uintptr_t>(Msel)) & 15) return DFLASH_ERR_INVALID_ARG;
-  const Layout lo = layout(L, r);
+  constexpr int OFF = WALK == WALK_VITERBI ? 0 : 1;
+  const int npairs = L + OFF - 1;
+  const Layout lo = layout(L + OFF, r);
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(path_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    attr_err =
+        cudaFuncSetAttribute(path_select_kernel<WALK>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
   });
   if (attr_err != cudaSuccess) return DFLASH_ERR_CUDA;
   // Few blocks: one cluster of up to 8 CTAs per block spreads its pair scoring
@@ -314,15 +433,14 @@ static int launch(const float* topk_logp, const int32_t* topk_idx, const dflash_
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   int Q = 1;
-  if (B * 2 < sms && L > 2) {
-    Q = L - 1 < MAX_CLUSTER ? L - 1 : MAX_CLUSTER;
+  if (B * 2 < sms && npairs > 1) {
+    Q = npairs < MAX_CLUSTER ? npairs : MAX_CLUSTER;
     while (Q > 1 && static_cast<long long>(B) * Q > sms) --Q;
   }
-  const cudaError_t e =
-      launch_kernel_cluster(path_select_kernel, dim3(B * Q), dim3(THREADS), lo.total, static_cast<cudaStream_t>(stream),
-                            Q, topk_logp, topk_idx, reinterpret_cast<const uint16_t*>(E),
-                            reinterpret_cast<const uint16_t*>(Msel), L, r, V, path_tok, path_slot, path_score,
-                            pair_scores_dbg, dev_status, target, accept_len, next_token, Q);
+  const cudaError_t e = launch_kernel_cluster(
+      path_select_kernel<WALK>, dim3(B * Q), dim3(THREADS), lo.total, static_cast<cudaStream_t>(stream), Q,
+      topk_logp, topk_idx, reinterpret_cast<const uint16_t*>(E), reinterpret_cast<const uint16_t*>(Msel), L, r, V,
+      path_tok, path_slot, path_score, pair_scores_dbg, dev_status, target, accept_len, next_token, Q, wa);
   return e == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }
 
@@ -333,8 +451,9 @@ extern "C" int dflash_path_select(const float* topk_logp, const int32_t* topk_id
                                   const dflash_bf16* Msel, int B, int L, int K, int r, int V, int32_t* path_tok,
                                   int32_t* path_slot, float* path_score, float* pair_scores_dbg, int* dev_status,
                                   void* stream) {
-  return dflash::sel::launch(topk_logp, topk_idx, E, Msel, B, L, K, r, V, path_tok, path_slot, path_score,
-                             pair_scores_dbg, nullptr, nullptr, nullptr, dev_status, stream);
+  return dflash::sel::launch<dflash::sel::WALK_VITERBI>(topk_logp, topk_idx, E, Msel, B, L, K, r, V, path_tok,
+                                                        path_slot, path_score, pair_scores_dbg, nullptr, nullptr,
+                                                        nullptr, dev_status, stream, dflash::sel::WalkArgs{});
 }
 
 extern "C" int dflash_select_verify(const float* topk_logp, const int32_t* topk_idx, const dflash_bf16* E,
@@ -342,6 +461,25 @@ extern "C" int dflash_select_verify(const float* topk_logp, const int32_t* topk_
                                     int V, int32_t* path_tok, int32_t* path_slot, float* path_score,
                                     int32_t* accept_len, int32_t* next_token, int* dev_status, void* stream) {
   if (!target || !accept_len || !next_token) return DFLASH_ERR_INVALID_ARG;
-  return dflash::sel::launch(topk_logp, topk_idx, E, Msel, B, L, K, r, V, path_tok, path_slot, path_score,
-                             nullptr, target, accept_len, next_token, dev_status, stream);
+  return dflash::sel::launch<dflash::sel::WALK_VITERBI>(topk_logp, topk_idx, E, Msel, B, L, K, r, V, path_tok,
+                                                        path_slot, path_score, nullptr, target, accept_len,
+                                                        next_token, dev_status, stream, dflash::sel::WalkArgs{});
+}
+
+extern "C" int dflash_path_walk(const float* topk_logp, const int32_t* topk_idx, const dflash_bf16* E,
+                                const dflash_bf16* Msel, const int32_t* anchor, const float* uniforms,
+                                float temperature, int B, int L, int K, int r, int V, int32_t* path_tok,
+                                int32_t* path_slot, float* path_score, float* path_q, const int32_t* target,
+                                int32_t* accept_len, int32_t* next_token, int* dev_status, void* stream) {
+  using namespace dflash::sel;
+  if (!anchor) return DFLASH_ERR_INVALID_ARG;
+  if (target && (!accept_len || !next_token)) return DFLASH_ERR_INVALID_ARG;
+  WalkArgs wa{anchor, uniforms, 0.f, path_q};
+  if (uniforms == nullptr)
+    return launch<WALK_GREEDY>(topk_logp, topk_idx, E, Msel, B, L, K, r, V, path_tok, path_slot, path_score, nullptr,
+                               target, accept_len, next_token, dev_status, stream, wa);
+  if (!(temperature > 0.f) || !(temperature < INFINITY)) return DFLASH_ERR_INVALID_ARG;
+  wa.inv_t = 1.f / temperature;
+  return launch<WALK_SAMPLE>(topk_logp, topk_idx, E, Msel, B, L, K, r, V, path_tok, path_slot, path_score, nullptr,
+                             target, accept_len, next_token, dev_status, stream, wa);
 }

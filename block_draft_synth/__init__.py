@@ -26,7 +26,7 @@ K_TOP = 16
 
 # Order of the per-array child streams; fixed so every array is reproducible.
 STREAMS = ("H", "W", "a0", "a1", "x_conv", "prev", "E", "M", "noise", "bonus",
-           "topk", "verify", "Wc", "gate")
+           "topk", "verify", "Wc", "gate", "anchor", "u_walk", "u_accept", "u_resample", "z_target")
 
 
 @dataclasses.dataclass(frozen=True)
@@ -196,3 +196,29 @@ def synthetic_verify(B: int, L: int, V: int, seed: int, p_match):
     target[:, :L] = np.where(hit, draft, other)
     target[:, L] = rng.integers(0, V, size=B)
     return draft.astype(np.int32), target.astype(np.int32)
+
+
+# --- inputs of the sampled walk and of rejection-sampling verification -------
+
+def anchors(B: int, V: int, seed: int) -> np.ndarray:
+    """The last verified token of each block, uniform over [0, V), int32 [B]."""
+    return rng_for(seed, "anchor").integers(0, V, size=B).astype(np.int32)
+
+
+def uniforms(shape, seed: int, stream: str) -> np.ndarray:
+    """fp32 uniforms in [0, 1) for one of the named draws ("u_walk",
+    "u_accept", "u_resample")."""
+    if stream not in ("u_walk", "u_accept", "u_resample"):
+        raise KeyError(stream)
+    u = rng_for(seed, stream).random(size=shape, dtype=np.float32)
+    return np.minimum(u, np.float32(1.0 - 2.0 ** -24))
+
+
+def target_logits(rows: int, V: int, seed: int, scale: float = 2.0) -> np.ndarray:
+    """A target model's logits for `rows` positions: fp32 N(0, scale^2) [rows, V]."""
+    rng = rng_for(seed, "z_target")
+    out = np.empty((rows, V), dtype=np.float32)
+    for r0 in range(0, rows, 64):
+        r1 = min(rows, r0 + 64)
+        out[r0:r1] = rng.standard_normal((r1 - r0, V), dtype=np.float32) * np.float32(scale)
+    return out

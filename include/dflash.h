@@ -7,6 +7,10 @@
  *                       log-softmax and per-position top-16 selection
  *   dflash_path_select  pair scores of neighbouring candidates + max-sum walk
  *   dflash_verify       greedy verification (accepted length, next token)
+ * and the walks and verification the pages describe beside the max-sum walk:
+ *   dflash_path_walk        greedy or sampled walk from the last verified token
+ *   dflash_verify_rejection rejection-sampling verification against the
+ *                           target's distributions
  *
  * Sources: "DFlash 2: Keep Drafting Parallel" (the blog, read in its Chinese
  * translation) and "Inco AI's DFlash 2 lifts LLM decoding output 16-25%".
@@ -203,6 +207,69 @@ int dflash_select_verify(const float* topk_logp, const int32_t* topk_idx, const 
                          const dflash_bf16* Msel, const int32_t* target, int B, int L, int K, int r, int V,
                          int32_t* path_tok, int32_t* path_slot, float* path_score, int32_t* accept_len,
                          int32_t* next_token, int* dev_status, void* stream);
+
+/*
+ * Walk from the last verified token.
+ * "DFlash 2: Keep Drafting Parallel", section "a lightweight path selector":
+ * starting from the last verified token, the walk over the precomputed pair
+ * scores greedily follows the best successor, or draws each successor from
+ * the same scores.  With the anchor a = anchor[b] and the stand-in scores
+ *   S_a[k]    = lp[b*L, k] + e_a . M . e_{c_0k}            (no unary term for a)
+ *   S_i[j,k]  = lp[b*L+i, j] + lp[b*L+i+1, k] + e_{c_ij} . M . e_{c_{i+1,k}}
+ * the walk picks slot s_0 from S_a and s_{i+1} from row S_i[s_i, :]:
+ *   uniforms == NULL  greedy: the argmax (ties: lowest slot);
+ *   otherwise         sampling: q = softmax(row / temperature) over the 16
+ *                     slots, s = the smallest slot whose cumulative q exceeds
+ *                     uniforms[b*L+i] (inverse CDF in slot order).
+ *
+ * topk_logp, topk_idx [B*L, 16] as from dflash_lmhead_topk; E [V, r] bf16,
+ * Msel [r, r] bf16 (16-byte aligned); anchor [B] int32; uniforms [B, L] fp32
+ * in [0, 1) or NULL; temperature > 0 (sampling only).
+ * Outputs: path_tok [B, L] int32; path_slot [B, L] int32 (nullable);
+ * path_score [B] fp32 (nullable; S_a[s_0] + sum_i S_i[s_i, s_{i+1}]);
+ * path_q [B, L, 16] fp32 (nullable; sampling only: the distribution each slot
+ * was drawn from, what dflash_verify_rejection needs as draft_q).
+ * target [B, L+1] int32 (nullable): if given, the path is verified greedily
+ * as dflash_verify does, into accept_len [B] and next_token [B].
+ * 1 <= L <= 16, 8 <= r <= 128, r % 8 == 0.  An anchor or candidate index
+ * outside [0, V) is read as 0 and records DFLASH_ERR_BAD_INDEX.
+ */
+int dflash_path_walk(const float* topk_logp, const int32_t* topk_idx, const dflash_bf16* E,
+                     const dflash_bf16* Msel, const int32_t* anchor, const float* uniforms,
+                     float temperature, int B, int L, int K, int r, int V, int32_t* path_tok,
+                     int32_t* path_slot, float* path_score, float* path_q, const int32_t* target,
+                     int32_t* accept_len, int32_t* next_token, int* dev_status, void* stream);
+
+/*
+ * Rejection-sampling verification of a sampled path.
+ * "DFlash 2: Keep Drafting Parallel", section "a lightweight path selector",
+ * and "Inco AI's DFlash 2 lifts LLM decoding output 16-25%": rejection
+ * sampling restores the target's exact output distribution.  Standard
+ * speculative sampling, with p_i = softmax(target_logits[b*(L+1)+i] / T) and
+ * q_i = draft_q[b*L+i] (on the candidates cand_idx[b*L+i]):
+ *   position i is kept while u_accept[b*L+i] * q_i[s_i] <= p_i(draft[b*L+i]);
+ *   with n the first rejected position (n = L if none), accept_len[b] = n + 1
+ *   and next_token[b] is drawn from max(0, p_n - q_n) (n < L) or from p_L
+ *   (n = L) by inverse CDF in vocabulary order: the smallest token whose
+ *   cumulative mass exceeds u_resample[b] times the total mass.
+ * The draw happens in fp64 on fp32 exponentials; a uniform that falls within
+ * about 1e-7 (relative) of a cumulative boundary may land on either side.
+ *
+ * target_logits [B*(L+1), V] fp32 (finite or -inf); temperature > 0 (the
+ * same one the draft was sampled at); draft, draft_slot [B, L] int32 (the
+ * path and its slots, as from dflash_path_walk); cand_idx [B*L, 16] int32
+ * (distinct per row); draft_q [B, L, 16] fp32; u_accept [B, L] and
+ * u_resample [B] fp32 uniforms in [0, 1).  accept_len, next_token [B] int32
+ * out.  ws: device workspace of dflash_verify_rejection_workspace(B, L, V)
+ * bytes, 16-byte aligned.  1 <= L <= 31, 1 <= V <= 524288.  A draft token or
+ * slot out of range records DFLASH_ERR_BAD_INDEX and is clamped.
+ */
+size_t dflash_verify_rejection_workspace(int B, int L, int V);
+int dflash_verify_rejection(const float* target_logits, float temperature, const int32_t* draft,
+                            const int32_t* draft_slot, const int32_t* cand_idx, const float* draft_q,
+                            const float* u_accept, const float* u_resample, int B, int L, int V,
+                            int32_t* accept_len, int32_t* next_token, void* ws, size_t ws_bytes,
+                            int* dev_status, void* stream);
 
 /*
  * Greedy verification.

@@ -41,8 +41,9 @@ from .conv import conv2tap, conv2tap_dynamic
 from .lmhead import logits, lmhead_topk, argmax_tokens, topk_margin_ok
 from .selector import pair_scores, viterbi, viterbi_two_best, path_select
 from .verify import verify
-from .walks import anchor_scores, greedy_walk, sample_walk, verify_rejection, inverse_cdf
+from .walks import anchor_scores, greedy_walk, sample_walk, verify_rejection, inverse_cdf, target_probs
 
 __all__ = ["conv2tap", "conv2tap_dynamic", "logits", "lmhead_topk", "argmax_tokens", "topk_margin_ok",
            "pair_scores", "viterbi", "viterbi_two_best", "path_select", "verify",
-           "anchor_scores", "greedy_walk", "sample_walk", "verify_rejection", "inverse_cdf"]
+           "anchor_scores", "greedy_walk", "sample_walk", "verify_rejection", "inverse_cdf",
+           "target_probs"]

@@ -116,6 +116,14 @@ def sample_walk(topk_logp, topk_idx, E_bits, M_bits, anchor, uniforms, T: float,
     return {"path_slot": slots, "path_tok": tok, "q": q, "gap": gap}
 
 
+def target_probs(z, T: float) -> np.ndarray:
+    """p = softmax(z / T) along the last axis, float64, from fp32 logits."""
+    x = np.asarray(z, dtype=np.float32).astype(np.float64) / T
+    x = x - x.max(axis=-1, keepdims=True)
+    e = np.exp(x)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
 def verify_rejection(draft, draft_slot, cand_idx, draft_q, target_p, u_accept, u_resample):
     """Speculative-sampling verification.
 

@@ -62,6 +62,27 @@ def test_host_side_rejections(lib):
     # verify: L out of range
     assert lib.dflash_verify(fake, fake, 1, 0, fake, fake, None) == 1
     assert lib.dflash_verify(fake, fake, 1, 33, fake, fake, None) == 1
+    # walk: no anchor; sampling at temperature 0; target without outputs
+    f32 = ctypes.c_float
+    lib.dflash_path_walk.argtypes = [vp, vp, vp, vp, vp, vp, f32] + [ctypes.c_int] * 5 + [vp] * 9
+    assert lib.dflash_path_walk(fake, fake, fake, fake, None, None, 1.0, 1, 4, 16, 32, 100,
+                                fake, None, None, None, None, None, None, None, None) == 1
+    assert lib.dflash_path_walk(fake, fake, fake, fake, fake, fake, 0.0, 1, 4, 16, 32, 100,
+                                fake, None, None, None, None, None, None, None, None) == 1
+    assert lib.dflash_path_walk(fake, fake, fake, fake, fake, None, 1.0, 1, 4, 16, 32, 100,
+                                fake, None, None, None, fake, None, None, None, None) == 1
+    # rejection verify: temperature <= 0, L > 31, V too large, workspace too small
+    lib.dflash_verify_rejection.argtypes = ([vp, f32] + [vp] * 6 + [ctypes.c_int] * 3 + [vp, vp, vp,
+                                            ctypes.c_size_t, vp, vp])
+    big = ctypes.c_size_t(1 << 30)
+    args = lambda T, B, L, V, ws: (fake, T, fake, fake, fake, fake, fake, fake, B, L, V, fake, fake, fake, ws,
+                                   None, None)
+    assert lib.dflash_verify_rejection(*args(0.0, 1, 4, 1000, big)) == 1
+    assert lib.dflash_verify_rejection(*args(1.0, 1, 32, 1000, big)) == 1
+    assert lib.dflash_verify_rejection(*args(1.0, 1, 4, 524289, big)) == 1
+    assert lib.dflash_verify_rejection(*args(1.0, 1, 4, 1000, ctypes.c_size_t(8))) == 4
+    lib.dflash_verify_rejection_workspace.restype = ctypes.c_size_t
+    assert lib.dflash_verify_rejection_workspace(2, 3, 8193) == 2 * 4 * 2 * 16
 
 
 def test_workspace_rejects_bad_sizes(lib):

@@ -244,3 +244,13 @@ def test_planted_residual_sign_error_is_caught():
         for ur in g:
             first[wrong_next(s, ur)] += q[s] * (1 - acc) / n
     assert np.abs(first - p[0]).max() > 10.0 / n
+
+
+def test_target_probs_closed_forms():
+    z = np.log(np.array([[1.0, 2.0, 3.0], [5.0, 5.0, 5.0]], dtype=np.float32))
+    p = oracle.target_probs(z, 1.0)
+    np.testing.assert_allclose(p[0], [1 / 6, 2 / 6, 3 / 6], rtol=1e-6)
+    np.testing.assert_allclose(p[1], [1 / 3] * 3, rtol=1e-15)
+    # temperature 2 on log-weights (1, 4, 9) gives weights (1, 2, 3)
+    z2 = np.log(np.array([[1.0, 4.0, 9.0]], dtype=np.float32))
+    np.testing.assert_allclose(oracle.target_probs(z2, 2.0)[0], [1 / 6, 2 / 6, 3 / 6], rtol=1e-6)

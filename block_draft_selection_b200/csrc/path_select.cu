@@ -99,16 +99,15 @@ struct WalkArgs {
 //   greedy: next = argmax_k S_i[cur, k] (ties: lowest k)
 //   sample: q = softmax(S_i[cur, :] / T); next = the smallest k whose
 //           cumulative q exceeds u_i (inverse CDF in slot order)
+// pre_t / pre_u: lane i holds target token i / uniform i (read earlier).
 template <int WALK>
 __device__ __forceinline__ void walk_from_anchor(const float* Ss, const int* toks, int L, int b, const WalkArgs& wa,
-                                                 int32_t* path_tok, int32_t* path_slot, float* path_score,
-                                                 const int32_t* target, int32_t* accept_len, int32_t* next_token) {
+                                                 int pre_t, float pre_u, int32_t* path_tok, int32_t* path_slot,
+                                                 float* path_score, bool verify, int32_t* accept_len,
+                                                 int32_t* next_token) {
   const int lane = threadIdx.x & 31;
   const int k = lane & 15;
   const size_t row0 = static_cast<size_t>(b) * L;
-  // the uniforms of this block, one per lane (read before the serial walk)
-  float u_mine = 0.f;
-  if (WALK == WALK_SAMPLE && lane < L) u_mine = __ldg(wa.uniforms + row0 + lane);
   int cur = 0;
   int my_slot = 0;  // lane i keeps the slot chosen at position i
   float score = 0.f;
@@ -141,7 +140,7 @@ __device__ __forceinline__ void walk_from_anchor(const float* Ss, const int* tok
         if (k >= off) c += t;
       }
       const float total = __shfl_sync(0xffffffffu, c, 15);
-      const float u = __shfl_sync(0xffffffffu, u_mine, i);
+      const float u = __shfl_sync(0xffffffffu, pre_u, i);
       const unsigned over = __ballot_sync(0xffffffffu, c > u * total) & 0xffffu;
       nk = over ? __ffs(over) - 1 : 15;
       if (wa.path_q && lane < 16) wa.path_q[(row0 + i) * KC + k] = e / total;
@@ -157,14 +156,14 @@ __device__ __forceinline__ void walk_from_anchor(const float* Ss, const int* tok
     if (path_slot) path_slot[row0 + lane] = my_slot;
   }
   if (path_score && lane == 0) path_score[b] = score;
-  if (target != nullptr) {
-    const int32_t* tg = target + static_cast<size_t>(b) * (L + 1);
-    const bool differs = in_block && my_tok != __ldg(tg + lane);
+  if (verify) {
+    const bool differs = in_block && my_tok != pre_t;
     const unsigned mask = __ballot_sync(0xffffffffu, differs);
     const int n = mask ? __ffs(mask) - 1 : L;
+    const int nt = __shfl_sync(0xffffffffu, pre_t, n);
     if (lane == 0) {
       accept_len[b] = n + 1;
-      next_token[b] = __ldg(tg + n);
+      next_token[b] = nt;
     }
   }
 }
@@ -197,6 +196,15 @@ __global__ void __launch_bounds__(THREADS) path_select_kernel(
   const int r8 = r / 8;
   const size_t row0 = static_cast<size_t>(b) * L;
   const int npos = Li - 1;  // pair tables
+  // The leader's warp 0 reads now what the walk and the verification need at
+  // the end (lane i: target token i, uniform i), so those loads overlap the
+  // scoring instead of following the walk.
+  int pre_t = 0;
+  float pre_u = 0.f;
+  if (q_rank == 0 && tid < 32) {
+    if (target != nullptr && tid <= L) pre_t = __ldg(target + static_cast<size_t>(b) * (L + 1) + tid);
+    if (WALK == WALK_SAMPLE && tid < L) pre_u = __ldg(wa.uniforms + row0 + tid);
+  }
   // Scores go to the leader's shared memory (this CTA's own when Q == 1).
   // The leader's shared memory may be written only once every CTA of the
   // cluster runs: arrive now, wait just before the first remote store.
@@ -262,19 +270,24 @@ __global__ void __launch_bounds__(THREADS) path_select_kernel(
   const int my_npos = npos > q_rank ? (npos - q_rank + Q - 1) / Q : 0;
   for (int m0 = 0; m0 < my_npos; m0 += lo.pc) {
     const int pcn = min(lo.pc, my_npos - m0);
-    // u[ii][j][t] = sum_s e_{c_(i0+ii),j}[s] * M[s][t], 8 outputs per item
-    for (int q = tid; q < pcn * KC * r8; q += nthr) {
-      const int tg = q % r8;
-      const int jj = q / r8;  // (ii * 16 + j)
+    // u[ii][j][t] = sum_s e_{c_(i0+ii),j}[s] * M[s][t], 8 outputs per item;
+    // neighbouring lanes take the two halves of the s range and add them with
+    // one shuffle (the item count is a multiple of 32: whole warps iterate)
+    const int rh = r / 2;
+    for (int q = tid; q < pcn * KC * r8 * 2; q += nthr) {
+      const int h = q & 1;
+      const int tg = (q >> 1) % r8;
+      const int jj = (q >> 1) / r8;  // (ii * 16 + j)
       const int ii = jj / KC;
       const int j = jj - ii * KC;
       const int i = q_rank + Q * (m0 + ii);
-      const uint16_t* er = Es + static_cast<size_t>(i * KC + j) * lo.rp;
+      const uint16_t* er = Es + static_cast<size_t>(i * KC + j) * lo.rp + h * rh;
+      const uint16_t* mr = Ms + static_cast<size_t>(h * rh) * r + tg * 8;
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
-      for (int s = 0; s < r; ++s) {
+      for (int s = 0; s < rh; ++s) {
         const float es = __uint_as_float(static_cast<uint32_t>(er[s]) << 16);
-        const uint4 mv = *reinterpret_cast<const uint4*>(Ms + static_cast<size_t>(s) * r + tg * 8);
+        const uint4 mv = *reinterpret_cast<const uint4*>(mr + static_cast<size_t>(s) * r);
         acc[0] = fmaf(es, bf_lo(mv.x), acc[0]);
         acc[1] = fmaf(es, bf_hi(mv.x), acc[1]);
         acc[2] = fmaf(es, bf_lo(mv.y), acc[2]);
@@ -284,9 +297,13 @@ __global__ void __launch_bounds__(THREADS) path_select_kernel(
         acc[6] = fmaf(es, bf_lo(mv.w), acc[6]);
         acc[7] = fmaf(es, bf_hi(mv.w), acc[7]);
       }
-      float* ur = Us + static_cast<size_t>(jj) * lo.up + tg * 8;
-      *reinterpret_cast<float4*>(ur) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      *reinterpret_cast<float4*>(ur + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], 1);
+      if (h == 0) {
+        float* ur = Us + static_cast<size_t>(jj) * lo.up + tg * 8;
+        *reinterpret_cast<float4*>(ur) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4*>(ur + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      }
     }
     __syncthreads();
     for (int q = tid; q < pcn * KC * KC; q += nthr) {
@@ -324,8 +341,9 @@ __global__ void __launch_bounds__(THREADS) path_select_kernel(
     if (q_rank != 0) return;
   }
   if (WALK != WALK_VITERBI) {
-    if (tid < 32) walk_from_anchor<WALK>(Ss, toks, L, b, wa, path_tok, path_slot, path_score, target, accept_len,
-                                         next_token);
+    if (tid < 32)
+      walk_from_anchor<WALK>(Ss, toks, L, b, wa, pre_t, pre_u, path_tok, path_slot, path_score, target != nullptr,
+                             accept_len, next_token);
     return;
   }
   if (tid < 32) {
@@ -390,13 +408,13 @@ __global__ void __launch_bounds__(THREADS) path_select_kernel(
     }
     // ---- 4. optional greedy verification of the selected path ------------
     if (target != nullptr) {
-      const int32_t* tg = target + static_cast<size_t>(b) * (L + 1);
-      const bool differs = in_block && my_tok != __ldg(tg + lane);
+      const bool differs = in_block && my_tok != pre_t;
       const unsigned mask = __ballot_sync(0xffffffffu, differs);
       const int n = mask ? __ffs(mask) - 1 : L;
+      const int nt = __shfl_sync(0xffffffffu, pre_t, n);
       if (lane == 0) {
         accept_len[b] = n + 1;
-        next_token[b] = __ldg(tg + n);
+        next_token[b] = nt;
       }
     }
   }

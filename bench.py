@@ -189,9 +189,17 @@ class ClockSampler:
 # --------------------------------------------------------------- GPU arm ----
 
 class Step:
-    """One draft cycle on device-resident buffers, through the C ABI."""
+    """One draft cycle on device-resident buffers, through the C ABI.
 
-    def __init__(self, w: syn.Workload, rank: int, device):
+    cycle "greedy": conv, LM head top-16, max-sum selection + greedy
+    verification (the path the metric names).  cycle "sample": conv, LM head
+    top-16, a sampled walk from the last verified token (T = 1) and
+    rejection-sampling verification against the target's logits (resident
+    on the device, as a target model leaves them)."""
+
+    TEMPERATURE = 1.0
+
+    def __init__(self, w: syn.Workload, rank: int, device, cycle: str = "greedy"):
         import torch
         import block_draft_selection_b200 as bds
         self.bds, self.torch, self.w = bds, torch, w
@@ -218,11 +226,31 @@ class Step:
         self.tok, self.slot = e((w.B, w.L), torch.int32), e((w.B, w.L), torch.int32)
         self.score, self.acc, self.nxt = e(w.B, torch.float32), e(w.B, torch.int32), e(w.B, torch.int32)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.cycle = cycle
+        if cycle == "sample":
+            # the target's logits at the L drafted positions and the bonus
+            # position (the library's plain GEMM on the noised hidden states)
+            self.z_target = bds.dflash_gemm_bf16(Hn, self.W)
+            self.anchor = torch.from_numpy(syn.anchors(w.B, w.V, wr.seed)).to(dev)
+            u = lambda shape, name: torch.from_numpy(syn.uniforms(shape, wr.seed, name)).to(dev)
+            self.u_walk, self.u_acc, self.u_res = u((w.B, w.L), "u_walk"), u((w.B, w.L), "u_accept"), u((w.B,), "u_resample")
+            self.q = e((w.B, w.L, 16), torch.float32)
+            self.rws = torch.empty(max(1, bds.dflash_verify_rejection_workspace(w.B, w.L, w.V)), dtype=torch.uint8,
+                                   device=dev)
 
     # conv, LM-head GEMM+epilogue, LM-head merge, select+verify
     LAUNCHES_PER_STEP = 4
     STAGES = ("conv2tap", "lmhead_topk", "select_verify")
-    TIMED = STAGES + ("event_pair",)
+    # "lmhead_select" brackets the LM head and the selection stage of one
+    # cycle together: minus the LM head's own bracket it is the time the
+    # selection stage adds to a cycle, with the selector's launch allowed to
+    # overlap the end of the LM head as it does in untimed cycles
+    TIMED = STAGES + ("event_pair", "lmhead_select")
+    # sample cycle: conv, LM head (2), walk, rejection verification (2)
+    LAUNCHES_PER_STEP_SAMPLE = 6
+
+    def launches(self):
+        return self.LAUNCHES_PER_STEP_SAMPLE if self.cycle == "sample" else self.LAUNCHES_PER_STEP
 
     def run(self, marks=None):
         """One cycle.  `marks`: optional {stage name: (event, event)} recorded
@@ -240,12 +268,28 @@ class Step:
 
         stage("event_pair", lambda: None)    # calibration: two event nodes, nothing between
         stage("conv2tap", lambda: bds.dflash_conv2tap(self.x, self.a0, self.a1, self.prev, y=self.y))
+        span = marks.get("lmhead_select")
+        if span:
+            span[0].record()
         stage("lmhead_topk", lambda: bds.dflash_lmhead_topk(
             self.H, self.W, topk_logp=self.lp, topk_idx=self.ix, lse=self.lse, ws=self.ws, dev_status=self.status))
-        stage("select_verify", lambda: bds.dflash_select_verify(
-            self.lp, self.ix, self.E, self.Msel, self.target, self.w.B, self.w.L, path_tok=self.tok,
-            path_slot=self.slot, path_score=self.score, accept_len=self.acc, next_token=self.nxt,
-            dev_status=self.status))
+        if self.cycle == "sample":
+            def walk_verify():
+                bds.dflash_path_walk(self.lp, self.ix, self.E, self.Msel, self.anchor, self.w.B, self.w.L,
+                                     uniforms=self.u_walk, temperature=self.TEMPERATURE, path_tok=self.tok,
+                                     path_slot=self.slot, path_score=self.score, path_q=self.q,
+                                     dev_status=self.status)
+                bds.dflash_verify_rejection(self.z_target, self.TEMPERATURE, self.tok, self.slot, self.ix, self.q,
+                                            self.u_acc, self.u_res, accept_len=self.acc, next_token=self.nxt,
+                                            ws=self.rws, dev_status=self.status)
+            stage("select_verify", walk_verify)
+        else:
+            stage("select_verify", lambda: bds.dflash_select_verify(
+                self.lp, self.ix, self.E, self.Msel, self.target, self.w.B, self.w.L, path_tok=self.tok,
+                path_slot=self.slot, path_score=self.score, accept_len=self.acc, next_token=self.nxt,
+                dev_status=self.status))
+        if span:
+            span[1].record()
 
 
 def _graph_steps(step, n_steps):
@@ -258,7 +302,7 @@ def _graph_steps(step, n_steps):
     ev = lambda: (torch.cuda.Event(enable_timing=True, external=True),
                   torch.cuda.Event(enable_timing=True, external=True))
     plan = {n_steps - 1: "lmhead_topk", n_steps - 2: "select_verify", n_steps - 3: "conv2tap",
-            n_steps - 4: "event_pair"}
+            n_steps - 4: "event_pair", n_steps - 5: "lmhead_select"}
     marks = {k: {name: ev()} for k, name in plan.items() if k >= 0}
     g = torch.cuda.CUDAGraph()
     side = torch.cuda.Stream()
@@ -291,7 +335,7 @@ def gpu_arm(args, w: syn.Workload):
                                 device_id=torch.device("cuda", local_rank))
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
-    step = Step(w, rank, device)
+    step = Step(w, rank, device, args.cycle)
 
     def barrier():
         torch.cuda.synchronize()
@@ -341,6 +385,10 @@ def gpu_arm(args, w: syn.Workload):
     stage_ms = [max(0.0, t - ev_ms) for t in raw_ms]
     lm_ms = raw_ms[1]                   # gross: includes the bracketing event nodes (conservative)
     lm_net_ms = stage_ms[1]
+    # time the selection stage adds to a cycle (both brackets gross, so the
+    # event-node cost cancels)
+    span_ms = mean("lmhead_select") if samples["lmhead_select"] else float("nan")
+    sel_added_ms = max(0.0, span_ms - lm_ms) if span_ms == span_ms else None
     ms_max = reduce_max(ms, world)
     value = aggregate(w.B, world, ms_max, args.steps)
     del graphs
@@ -348,26 +396,34 @@ def gpu_arm(args, w: syn.Workload):
     # end-to-end leg: the library's DraftCycle, one graph launch per step that
     # copies the step's inputs from pinned host memory, runs the cycle and
     # copies the results back; the host waits for them every step
-    cyc = bds.DraftCycle(step.W, step.E, step.Msel, step.a0, step.a1, w.B, w.L, w.P)
-    cyc.host_in["H"].copy_(step.H)
-    cyc.host_in["x"].copy_(step.x)
-    cyc.host_in["prev"].copy_(step.prev)
-    cyc.host_in["target"].copy_(step.target)
-    for _ in range(max(3, args.warmup // 2)):
-        cyc.run()
-    barrier()
-    e_steps = max(1, args.steps)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(e_steps):
-        cyc.run()
-    e1.record()
-    torch.cuda.synchronize()
-    barrier()
-    if int(cyc.status.item()) != 0:
-        raise RuntimeError(f"device status {int(cyc.status.item())} in the end-to-end leg")
-    e_ms = reduce_max(e0.elapsed_time(e1), world)
-    h2d, d2h = cyc.io_bytes()
+    e2e = None
+    if args.cycle == "greedy":
+        cyc = bds.DraftCycle(step.W, step.E, step.Msel, step.a0, step.a1, w.B, w.L, w.P)
+        cyc.host_in["H"].copy_(step.H)
+        cyc.host_in["x"].copy_(step.x)
+        cyc.host_in["prev"].copy_(step.prev)
+        cyc.host_in["target"].copy_(step.target)
+        for _ in range(max(3, args.warmup // 2)):
+            cyc.run()
+        barrier()
+        e_steps = max(1, args.steps)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(e_steps):
+            cyc.run()
+        e1.record()
+        torch.cuda.synchronize()
+        barrier()
+        if int(cyc.status.item()) != 0:
+            raise RuntimeError(f"device status {int(cyc.status.item())} in the end-to-end leg")
+        e_ms = reduce_max(e0.elapsed_time(e1), world)
+        h2d, d2h = cyc.io_bytes()
+        e2e = {"value": aggregate(w.B, world, e_ms, e_steps), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "path": "DraftCycle.run(): pinned H2D + conv + LM head + select/verify + D2H, host sync"}
+    else:
+        e2e = {"value": None, "unit": UNIT, "h2d_bytes_per_step": None, "d2h_bytes_per_step": None,
+               "path": "not measured for the sampled cycle: its target logits live on the device"}
 
     peaks, peaks_kind = load_peaks()
     alg_bytes, alg_flops = lmhead_algorithmic(w)
@@ -400,21 +456,27 @@ def gpu_arm(args, w: syn.Workload):
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded block_draft_synth; random-init weights of the workload's shapes)",
-            "config": {"workload": w.name, "blocks_per_gpu": w.B, "L": w.L, "M": w.M, "d": w.d, "V": w.V,
+            "config": {"workload": w.name if args.cycle == "greedy" else f"{w.name}+sampled-walk(T=1)",
+                       "blocks_per_gpu": w.B, "L": w.L, "M": w.M, "d": w.d, "V": w.V,
                        "K": 16, "r": w.r, "conv": [w.B, w.P, w.d], "parallelism": f"dp{world} (blocks)",
+                       "cycle": args.cycle,
                        "launch": "eager" if args.eager else f"cuda graphs of {chunk} cycles, PDL between kernels",
                        "l2": "inputs larger than L2 (W is %.0f MB > 126 MB)" % (2 * w.V * w.d / 1e6)},
-            "e2e": {"value": aggregate(w.B, world, e_ms, e_steps), "unit": UNIT,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "path": "DraftCycle.run(): pinned H2D + conv + LM head + select/verify + D2H, host sync"},
-            "gpu_launches": Step.LAUNCHES_PER_STEP * args.steps,
+            "e2e": e2e,
+            "gpu_launches": step.launches() * args.steps,
             "roofline": roof,
             "stages_us": {**{n: 1e3 * t for n, t in zip(Step.STAGES, stage_ms)},
                           "select_verify_share": stage_ms[2] / (ms_max / args.steps),
+                          "select_verify_added": None if sel_added_ms is None else 1e3 * sel_added_ms,
+                          "select_verify_added_share": (None if sel_added_ms is None
+                                                        else sel_added_ms / (ms_max / args.steps)),
                           "event_pair_overhead": 1e3 * ev_ms,
                           "raw": {n: 1e3 * t for n, t in zip(Step.STAGES, raw_ms)},
                           "samples": len(samples["lmhead_topk"]),
-                          "note": "durations net of the bracketing event-node pair (measured alone, 'raw' is gross)"},
+                          "note": ("durations net of the bracketing event-node pair (measured alone, 'raw' is "
+                                   "gross); select_verify_added = (LM head + selection bracketed together) - "
+                                   "(LM head bracketed alone): what the selection stage adds to a cycle when "
+                                   "its launch may overlap the LM head's end")},
             "clocks": clk.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -541,6 +603,9 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch each cycle eagerly instead of a CUDA graph")
+    ap.add_argument("--cycle", default="greedy", choices=["greedy", "sample"],
+                    help="greedy: max-sum selection + greedy verification (the metric's path); sample: "
+                         "sampled walk from the last verified token + rejection-sampling verification")
     ap.add_argument("--ref-budget-s", type=float, default=120.0,
                     help="host seconds the --impl reference run aims to take")
     args = ap.parse_args(argv)

@@ -62,7 +62,7 @@ __host__ __device__ inline Layout layout(int L, int r) {
   o.pc = pc;
   size_t off = 0;
   o.m_off = off;
-  off += static_cast<size_t>(r) * r * 2;
+  off += static_cast<size_t>(r) * o.rp * 2;  // M, or its transpose with padded rows (tensor-core path)
   off = (off + 15) & ~size_t(15);
   o.e_off = off;
   off += static_cast<size_t>(L) * KC * o.rp * 2;
@@ -82,6 +82,17 @@ __host__ __device__ inline Layout layout(int L, int r) {
 }
 
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+
+// d += A (16x16, row-major, bf16) . B (16x8, column-major, bf16), fp32
+// accumulate; fragments in the standard m16n8k16 register layout.
+__device__ __forceinline__ void mma_bf16_m16n8k16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                                  uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
 enum Walk { WALK_VITERBI = 0, WALK_GREEDY = 1, WALK_SAMPLE = 2 };
@@ -247,10 +258,25 @@ __global__ void __launch_bounds__(THREADS) path_select_kernel(
     }
     toks[q] = c;
   }
+  const bool use_mma = (r % 16) == 0;
   {
     const uint4* Mg = reinterpret_cast<const uint4*>(Msel);
-    uint4* Mv = reinterpret_cast<uint4*>(Ms);
-    for (int q = tid; q < r * r8; q += nthr) Mv[q] = __ldg(Mg + q);
+    if (use_mma) {
+      // transposed, rows padded to rp: column t of M is row t here, so the
+      // tensor-core B fragments are 32-bit loads without bank conflicts
+      for (int q = tid; q < r * r8; q += nthr) {
+        const int srow = q / r8;
+        const int c8 = q - srow * r8;
+        const uint4 v = __ldg(Mg + q);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          Ms[static_cast<size_t>(c8 * 8 + e) * lo.rp + srow] = static_cast<uint16_t>(w[e >> 1] >> (16 * (e & 1)));
+      }
+    } else {
+      uint4* Mv = reinterpret_cast<uint4*>(Ms);
+      for (int q = tid; q < r * r8; q += nthr) Mv[q] = __ldg(Mg + q);
+    }
   }
   for (int q = tid; q < Li * KC * r8; q += nthr) {
     const int cand = q / r8;
@@ -270,9 +296,39 @@ __global__ void __launch_bounds__(THREADS) path_select_kernel(
   const int my_npos = npos > q_rank ? (npos - q_rank + Q - 1) / Q : 0;
   for (int m0 = 0; m0 < my_npos; m0 += lo.pc) {
     const int pcn = min(lo.pc, my_npos - m0);
-    // u[ii][j][t] = sum_s e_{c_(i0+ii),j}[s] * M[s][t], 8 outputs per item;
-    // neighbouring lanes take the two halves of the s range and add them with
-    // one shuffle (the item count is a multiple of 32: whole warps iterate)
+    // u[ii][j][t] = sum_s e_{c_(i0+ii),j}[s] * M[s][t]
+    if (use_mma) {
+      // On the tensor cores: for each position, u (16 x r) = E rows (16 x r)
+      // . M (r x r) as mma.sync m16n8k16 (bf16 in, fp32 accumulate; the
+      // products are exact, as on the CUDA cores).  One warp per (position,
+      // 8-column n-tile).
+      const int warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
+      const int ntiles = r / 8;
+      for (int item = warp; item < pcn * ntiles; item += nthr / 32) {
+        const int ii = item / ntiles;
+        const int nt = item - ii * ntiles;
+        const int i = q_rank + Q * (m0 + ii);
+        const uint16_t* e0 = Es + static_cast<size_t>(i * KC + gq) * lo.rp + 2 * tq;
+        const uint16_t* e8 = e0 + 8 * lo.rp;
+        const uint16_t* mt = Ms + static_cast<size_t>(nt * 8 + gq) * lo.rp + 2 * tq;
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int k0 = 0; k0 < r; k0 += 16) {
+          const uint32_t a0 = *reinterpret_cast<const uint32_t*>(e0 + k0);
+          const uint32_t a1 = *reinterpret_cast<const uint32_t*>(e8 + k0);
+          const uint32_t a2 = *reinterpret_cast<const uint32_t*>(e0 + k0 + 8);
+          const uint32_t a3 = *reinterpret_cast<const uint32_t*>(e8 + k0 + 8);
+          const uint32_t b0 = *reinterpret_cast<const uint32_t*>(mt + k0);
+          const uint32_t b1 = *reinterpret_cast<const uint32_t*>(mt + k0 + 8);
+          mma_bf16_m16n8k16(d, a0, a1, a2, a3, b0, b1);
+        }
+        float* u0 = Us + static_cast<size_t>(ii * KC + gq) * lo.up + nt * 8 + 2 * tq;
+        *reinterpret_cast<float2*>(u0) = make_float2(d[0], d[1]);
+        *reinterpret_cast<float2*>(u0 + 8 * lo.up) = make_float2(d[2], d[3]);
+      }
+    } else {
+    // on the CUDA cores, 8 outputs per item; neighbouring lanes take the two
+    // halves of the s range and add them with one shuffle (the item count is
+    // a multiple of 32: whole warps iterate)
     const int rh = r / 2;
     for (int q = tid; q < pcn * KC * r8 * 2; q += nthr) {
       const int h = q & 1;
@@ -304,6 +360,7 @@ __global__ void __launch_bounds__(THREADS) path_select_kernel(
         *reinterpret_cast<float4*>(ur) = make_float4(acc[0], acc[1], acc[2], acc[3]);
         *reinterpret_cast<float4*>(ur + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
       }
+    }
     }
     __syncthreads();
     for (int q = tid; q < pcn * KC * KC; q += nthr) {

@@ -32,6 +32,11 @@ Pins (``tests/test_oracle_*.py``, run with ``-m "not gpu"``):
                 (= greedy), the E = 0 closed form at T = 1 (the renormalised
                 top-16), and the path distribution integrated over a grid of
                 uniforms against exact conditional softmaxes
+  ctx_tables / ctx_select (the pages' context-gated scorer)
+                a hand-worked case, exact rational tables with the gate
+                fixed at 1/2 and at 1, brute force over all 16^L anchored
+                paths, zero projections (= top-1 path), a planted swap of
+                the two projections
   verify_rejection
                 hand cases, and the output-distribution theorem: the first
                 emitted token is distributed exactly as the target's p_0
@@ -41,9 +46,10 @@ from .conv import conv2tap, conv2tap_dynamic
 from .lmhead import logits, lmhead_topk, argmax_tokens, topk_margin_ok
 from .selector import pair_scores, viterbi, viterbi_two_best, path_select
 from .verify import verify
+from .ctx_scorer import ctx_tables, ctx_select, maxsum_walk_tables
 from .walks import anchor_scores, greedy_walk, sample_walk, verify_rejection, inverse_cdf, target_probs
 
 __all__ = ["conv2tap", "conv2tap_dynamic", "logits", "lmhead_topk", "argmax_tokens", "topk_margin_ok",
            "pair_scores", "viterbi", "viterbi_two_best", "path_select", "verify",
            "anchor_scores", "greedy_walk", "sample_walk", "verify_rejection", "inverse_cdf",
-           "target_probs"]
+           "target_probs", "ctx_tables", "ctx_select", "maxsum_walk_tables"]

@@ -43,12 +43,25 @@ def anchor_scores(topk_logp, topk_idx, E_bits, M_bits, anchor, B: int, L: int) -
     return lp[:, 0, :] + np.einsum("br,bkr->bk", u, e0)
 
 
-def greedy_walk(topk_logp, topk_idx, E_bits, M_bits, anchor, B: int, L: int):
-    """Returns a dict: path_slot [B,L], path_tok [B,L], path_score [B] and
-    margin [B,L], the gap between the chosen and the runner-up score at each
-    step (0 where two candidates tie)."""
+def standin_anchored_tables(topk_logp, topk_idx, E_bits, M_bits, anchor, B: int, L: int) -> np.ndarray:
+    """Tables [B, L, K, K] of the walk from the anchor with the stand-in
+    scorer: table 0 holds S_a in every row (the anchor is one state), table
+    i >= 1 is the pair table S_{i-1} between drafted positions i-1 and i."""
     Sa = anchor_scores(topk_logp, topk_idx, E_bits, M_bits, anchor, B, L)
     S = pair_scores(topk_logp, topk_idx, E_bits, M_bits, B, L)
+    K = Sa.shape[1]
+    T = np.empty((B, L, K, K))
+    T[:, 0] = Sa[:, None, :]
+    T[:, 1:] = S
+    return T
+
+
+def greedy_walk_tables(T, topk_idx, B: int, L: int):
+    """Greedy walk over anchored tables T [B, L, K, K] (table 0's rows are the
+    anchor's): s_0 = argmax_k T_0[0, k], s_{i+1} = argmax_k T_{i+1}[s_i, k],
+    ties to the lowest slot.  Returns a dict: path_slot, path_tok [B, L],
+    path_score [B] (the sum of the chosen entries) and margin [B, L] (chosen
+    minus runner-up at each step)."""
     idx = np.asarray(topk_idx, dtype=np.int64).reshape(B, L, -1)
     slots = np.zeros((B, L), dtype=np.int64)
     score = np.zeros(B)
@@ -59,18 +72,23 @@ def greedy_walk(topk_logp, topk_idx, E_bits, M_bits, anchor, B: int, L: int):
         return row[k] - rest.max() if rest.size else np.inf
 
     for b in range(B):
-        k = int(np.argmax(Sa[b]))                          # first max = lowest slot
-        slots[b, 0] = k
-        score[b] = Sa[b, k]
-        margin[b, 0] = second_gap(Sa[b], k)
-        for i in range(L - 1):
-            nk = int(np.argmax(S[b, i, k]))
-            score[b] += S[b, i, k, nk]
-            margin[b, i + 1] = second_gap(S[b, i, k], nk)
-            k = nk
-            slots[b, i + 1] = k
+        cur = 0
+        for i in range(L):
+            row = T[b, i, cur]
+            k = int(np.argmax(row))                        # first max = lowest slot
+            score[b] += row[k]
+            margin[b, i] = second_gap(row, k)
+            slots[b, i] = k
+            cur = k
     tok = np.take_along_axis(idx, slots[:, :, None], axis=2)[:, :, 0]
     return {"path_slot": slots, "path_tok": tok, "path_score": score, "margin": margin}
+
+
+def greedy_walk(topk_logp, topk_idx, E_bits, M_bits, anchor, B: int, L: int):
+    """Greedy walk from the anchor with the stand-in scorer; see
+    greedy_walk_tables for the returned dict."""
+    T = standin_anchored_tables(topk_logp, topk_idx, E_bits, M_bits, anchor, B, L)
+    return greedy_walk_tables(T, topk_idx, B, L)
 
 
 def softmax_t(scores: np.ndarray, T: float) -> np.ndarray:
@@ -88,13 +106,13 @@ def inverse_cdf(prob: np.ndarray, u: float) -> int:
     return min(k, len(prob) - 1)
 
 
-def sample_walk(topk_logp, topk_idx, E_bits, M_bits, anchor, uniforms, T: float, B: int, L: int):
-    """Returns a dict: path_slot [B,L], path_tok [B,L], q [B,L,K] (q[b,i] is
-    the distribution the slot at position i was drawn from) and gap [B,L],
-    the distance of each uniform to the nearest inner cumulative-probability
+def sample_walk_tables(T, topk_idx, uniforms, temp: float, B: int, L: int):
+    """Sampled walk over anchored tables T [B, L, K, K]: the slot at position
+    i is drawn from softmax(T_i[s_{i-1}, :] / temp) (s_{-1} = 0, the anchor)
+    by inverse CDF with uniforms[b, i].  Returns a dict: path_slot, path_tok
+    [B, L], q [B, L, K] (the distribution each slot was drawn from) and gap
+    [B, L], the distance of each uniform to the nearest inner cumulative
     boundary (how close each draw came to changing)."""
-    Sa = anchor_scores(topk_logp, topk_idx, E_bits, M_bits, anchor, B, L)
-    S = pair_scores(topk_logp, topk_idx, E_bits, M_bits, B, L)
     idx = np.asarray(topk_idx, dtype=np.int64).reshape(B, L, -1)
     K = idx.shape[2]
     u = np.asarray(uniforms, dtype=np.float64).reshape(B, L)
@@ -102,18 +120,24 @@ def sample_walk(topk_logp, topk_idx, E_bits, M_bits, anchor, uniforms, T: float,
     q = np.zeros((B, L, K))
     gap = np.zeros((B, L))
     for b in range(B):
-        scores = Sa[b]
+        cur = 0
         for i in range(L):
-            pr = softmax_t(scores, T)
+            pr = softmax_t(T[b, i, cur], temp)
             k = inverse_cdf(pr, u[b, i])
             c = np.cumsum(pr)
             gap[b, i] = np.min(np.abs(c[:-1] - u[b, i])) if K > 1 else 1.0
             slots[b, i] = k
             q[b, i] = pr
-            if i + 1 < L:
-                scores = S[b, i, k]
+            cur = k
     tok = np.take_along_axis(idx, slots[:, :, None], axis=2)[:, :, 0]
     return {"path_slot": slots, "path_tok": tok, "q": q, "gap": gap}
+
+
+def sample_walk(topk_logp, topk_idx, E_bits, M_bits, anchor, uniforms, T: float, B: int, L: int):
+    """Sampled walk from the anchor with the stand-in scorer; see
+    sample_walk_tables for the returned dict."""
+    tables = standin_anchored_tables(topk_logp, topk_idx, E_bits, M_bits, anchor, B, L)
+    return sample_walk_tables(tables, topk_idx, uniforms, T, B, L)
 
 
 def target_probs(z, T: float) -> np.ndarray:

@@ -14,6 +14,9 @@ from ._binding import (  # noqa: F401
     LIB_PATH,
     dflash_conv2tap,
     dflash_conv2tap_dynamic,
+    dflash_ctx_project,
+    dflash_ctx_project_workspace,
+    dflash_ctx_walk,
     dflash_gemm_bf16,
     dflash_lmhead_logits_debug,
     dflash_lmhead_topk,

@@ -55,6 +55,10 @@ def _load():
         "dflash_path_walk": (i32, [vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, i32, i32, i32, i32,
                                    vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "dflash_verify_rejection_workspace": (sz, [i32, i32, i32]),
+        "dflash_ctx_project_workspace": (sz, [i32, i32, i32]),
+        "dflash_ctx_project": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, sz, vp, vp]),
+        "dflash_ctx_walk": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, ctypes.c_float,
+                                  vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "dflash_verify_rejection": (i32, [vp, ctypes.c_float, vp, vp, vp, vp, vp, vp, i32, i32, i32,
                                           vp, vp, vp, sz, vp, vp]),
     }
@@ -341,3 +345,69 @@ def dflash_verify_rejection(target_logits, temperature, draft, draft_slot, cand_
         _ptr(draft_q), _ptr(u_accept), _ptr(u_resample), B, L, V, _ptr(accept_len), _ptr(next_token),
         _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream)))
     return accept_len, next_token
+
+
+def dflash_ctx_project_workspace(B: int, L: int, d: int) -> int:
+    return int(lib.dflash_ctx_project_workspace(B, L, d))
+
+
+def dflash_ctx_project(Emb, H, Pab, Pg, topk_idx, anchor, B, L, proj=None, gate=None, ws=None, dev_status=None,
+                       stream=None):
+    """Projections of the context-gated scorer: returns (proj [B*(1+16L), 2e] f32,
+    gate [B*L, e] f32, before the sigmoid)."""
+    _need(Emb, "Emb", torch.bfloat16)
+    V, d = Emb.shape
+    _need(H, "H", torch.bfloat16, (B * L, d))
+    _need(Pab, "Pab", torch.bfloat16)
+    e = Pab.shape[0] // 2
+    _need(Pab, "Pab", torch.bfloat16, (2 * e, d))
+    _need(Pg, "Pg", torch.bfloat16, (e, d))
+    _need(topk_idx, "topk_idx", torch.int32, (B * L, K_TOP))
+    _need(anchor, "anchor", torch.int32, (B,))
+    dev = Emb.device
+    proj = _out(proj, "proj", torch.float32, (B * (1 + K_TOP * L), 2 * e), dev)
+    gate = _out(gate, "gate", torch.float32, (B * L, e), dev)
+    if ws is None:
+        ws = torch.empty(max(16, dflash_ctx_project_workspace(B, L, d)), dtype=torch.uint8, device=dev)
+    _check("dflash_ctx_project", lib.dflash_ctx_project(
+        _ptr(Emb), _ptr(H), _ptr(Pab), _ptr(Pg), _ptr(topk_idx), _ptr(anchor), B, L, V, d, e, _ptr(proj),
+        _ptr(gate), _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream)))
+    return proj, gate
+
+
+_WALKS = {"maxsum": 0, "greedy": 1, "sample": 2}
+
+
+def dflash_ctx_walk(topk_logp, topk_idx, anchor, proj, gate, B, L, V, walk="maxsum", uniforms=None,
+                    temperature=1.0, want_tables=False, target=None, path_tok=None, path_slot=None,
+                    path_score=None, path_q=None, accept_len=None, next_token=None, dev_status=None, stream=None):
+    """Scores of the context-gated scorer and a walk from the anchor.  Returns
+    (path_tok, path_slot, path_score, path_q or None, tables or None,
+    accept_len or None, next_token or None)."""
+    _need(topk_logp, "topk_logp", torch.float32, (B * L, K_TOP))
+    _need(topk_idx, "topk_idx", torch.int32, (B * L, K_TOP))
+    _need(anchor, "anchor", torch.int32, (B,))
+    _need(gate, "gate", torch.float32)
+    e = gate.shape[1]
+    _need(gate, "gate", torch.float32, (B * L, e))
+    _need(proj, "proj", torch.float32, (B * (1 + K_TOP * L), 2 * e))
+    dev = proj.device
+    if walk == "sample":
+        _need(uniforms, "uniforms", torch.float32, (B, L))
+    path_tok = _out(path_tok, "path_tok", torch.int32, (B, L), dev)
+    path_slot = _out(path_slot, "path_slot", torch.int32, (B, L), dev)
+    path_score = _out(path_score, "path_score", torch.float32, (B,), dev)
+    path_q = _out(path_q, "path_q", torch.float32, (B, L, K_TOP), dev) if walk == "sample" else None
+    tables = torch.empty((B, L, K_TOP, K_TOP), dtype=torch.float32, device=dev) if want_tables else None
+    if target is not None:
+        _need(target, "target", torch.int32, (B, L + 1))
+        accept_len = _out(accept_len, "accept_len", torch.int32, (B,), dev)
+        next_token = _out(next_token, "next_token", torch.int32, (B,), dev)
+    else:
+        accept_len = next_token = None
+    _check("dflash_ctx_walk", lib.dflash_ctx_walk(
+        _ptr(topk_logp), _ptr(topk_idx), _ptr(anchor), _ptr(proj), _ptr(gate), B, L, K_TOP, e, V, _WALKS[walk],
+        _ptr(uniforms) if walk == "sample" else None, float(temperature), _ptr(path_tok), _ptr(path_slot),
+        _ptr(path_score), _ptr(path_q), _ptr(tables), _ptr(target), _ptr(accept_len), _ptr(next_token),
+        _ptr(dev_status), _stream(stream)))
+    return path_tok, path_slot, path_score, path_q, tables, accept_len, next_token

@@ -26,7 +26,8 @@ K_TOP = 16
 
 # Order of the per-array child streams; fixed so every array is reproducible.
 STREAMS = ("H", "W", "a0", "a1", "x_conv", "prev", "E", "M", "noise", "bonus",
-           "topk", "verify", "Wc", "gate", "anchor", "u_walk", "u_accept", "u_resample", "z_target")
+           "topk", "verify", "Wc", "gate", "anchor", "u_walk", "u_accept", "u_resample", "z_target",
+           "Pab", "Pg")
 
 
 @dataclasses.dataclass(frozen=True)
@@ -222,3 +223,14 @@ def target_logits(rows: int, V: int, seed: int, scale: float = 2.0) -> np.ndarra
         r1 = min(rows, r0 + 64)
         out[r0:r1] = rng.standard_normal((r1 - r0, V), dtype=np.float32) * np.float32(scale)
     return out
+
+
+def ctx_scorer_weights(w: Workload, e: int = 256, scale: float = 0.2):
+    """Weights of the context-gated pair scorer: Pab [2e, d] ~ N(0, scale^2)
+    (the A and B projections of a token embedding; with the tied embedding
+    table = the LM head, N(0, 1/d), A and B are about N(0, scale^2)) and the
+    gate projection Pg [e, d] ~ N(0, 1/d) (a gate input of about N(0, 1) for
+    unit-variance hidden states).  bf16."""
+    Pab = _normal_bf16(rng_for(w.seed, "Pab"), (2 * e, w.d), scale)
+    Pg = _normal_bf16(rng_for(w.seed, "Pg"), (e, w.d), 1.0 / np.sqrt(w.d))
+    return Pab, Pg

@@ -42,17 +42,17 @@ def ctx_tables(topk_logp, topk_idx, Emb_bits, H_bits, Pab_bits, Pg_bits, anchor,
     lp = f32(topk_logp).reshape(B, L, -1)
     idx = np.asarray(topk_idx, dtype=np.int64).reshape(B, L, -1)
     K = lp.shape[2]
-    Emb = bf16(Emb_bits)
+    Emb_bits = np.asarray(Emb_bits)
     H = bf16(H_bits).reshape(B, L, -1)
     Pab = bf16(Pab_bits)
     e = Pab.shape[0] // 2
     Pa, Pb = Pab[:e], Pab[e:]
     Pg = bf16(Pg_bits)
     gate = sigmoid(H @ Pg.T)                               # [B, L, e]
-    cand = Emb[idx]                                        # [B, L, K, d]
+    cand = bf16(Emb_bits[idx])                             # [B, L, K, d]
     A_c = cand @ Pa.T                                      # [B, L, K, e]
     B_c = cand @ Pb.T                                      # [B, L, K, e]
-    A_anchor = Emb[np.asarray(anchor, dtype=np.int64)] @ Pa.T   # [B, e]
+    A_anchor = bf16(Emb_bits[np.asarray(anchor, dtype=np.int64)]) @ Pa.T   # [B, e]
     T = np.empty((B, L, K, K))
     for t in range(L):
         pred = A_anchor[:, None, :].repeat(K, axis=1) if t == 0 else A_c[:, t - 1]   # [B, K, e]

@@ -83,6 +83,24 @@ def test_host_side_rejections(lib):
     assert lib.dflash_verify_rejection(*args(1.0, 1, 4, 1000, ctypes.c_size_t(8))) == 4
     lib.dflash_verify_rejection_workspace.restype = ctypes.c_size_t
     assert lib.dflash_verify_rejection_workspace(2, 3, 8193) == 2 * 4 * 2 * 16
+    # context-gated scorer: e not a multiple of 8, L > 16, K != 16, unknown walk, sampling without uniforms
+    i32 = ctypes.c_int
+    lib.dflash_ctx_project.argtypes = [vp] * 6 + [i32] * 5 + [vp, vp, vp, ctypes.c_size_t, vp, vp]
+    assert lib.dflash_ctx_project(fake, fake, fake, fake, fake, fake, 1, 4, 100, 256, 20, fake, fake, fake, big,
+                                  None, None) == 1
+    assert lib.dflash_ctx_project(fake, fake, fake, fake, fake, fake, 1, 17, 100, 256, 32, fake, fake, fake, big,
+                                  None, None) == 1
+    assert lib.dflash_ctx_project(fake, fake, fake, fake, fake, fake, 1, 4, 100, 256, 32, fake, fake, fake,
+                                  ctypes.c_size_t(16), None, None) == 4
+    lib.dflash_ctx_project_workspace.restype = ctypes.c_size_t
+    assert lib.dflash_ctx_project_workspace(2, 3, 64) == 2 * 49 * 64 * 2
+    lib.dflash_ctx_walk.argtypes = [vp] * 5 + [i32] * 6 + [vp, f32] + [vp] * 10
+    walk = lambda K, walkid, u, T: lib.dflash_ctx_walk(fake, fake, fake, fake, fake, 1, 4, K, 32, 100, walkid, u, T,
+                                                       fake, None, None, None, None, None, None, None, None, None)
+    assert walk(8, 0, None, 1.0) == 1
+    assert walk(16, 3, None, 1.0) == 1
+    assert walk(16, 2, None, 1.0) == 1
+    assert walk(16, 2, fake, 0.0) == 1
 
 
 def test_workspace_rejects_bad_sizes(lib):

@@ -25,6 +25,9 @@ from ._binding import (  # noqa: F401
     dflash_path_walk,
     dflash_select_verify,
     dflash_lmhead_topk_static,
+    dflash_lmhead_topk_merge,
+    dflash_lmhead_topk_partial,
+    dflash_lmhead_topk_records,
     dflash_status_string,
     dflash_verify,
     dflash_verify_rejection,
@@ -33,6 +36,7 @@ from ._binding import (  # noqa: F401
     workspace,
 )
 from .cycle import DraftCycle  # noqa: F401,E402
+from .parallel import VocabParallelLMHead, vocab_shard  # noqa: F401,E402
 
 
 def bf16_tensor(bits: np.ndarray, device="cuda") -> torch.Tensor:

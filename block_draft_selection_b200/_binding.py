@@ -56,6 +56,9 @@ def _load():
                                    vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "dflash_verify_rejection_workspace": (sz, [i32, i32, i32]),
         "dflash_ctx_project_workspace": (sz, [i32, i32, i32]),
+        "dflash_lmhead_topk_records": (i32, [i32, i32, i32]),
+        "dflash_lmhead_topk_partial": (i32, [vp, vp, i32, i32, i32, i32, vp, sz, vp, vp]),
+        "dflash_lmhead_topk_merge": (i32, [vp, i32, i32, i32, i32, vp, vp, vp, vp]),
         "dflash_ctx_project": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, sz, vp, vp]),
         "dflash_ctx_walk": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, ctypes.c_float,
                                   vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
@@ -411,3 +414,43 @@ def dflash_ctx_walk(topk_logp, topk_idx, anchor, proj, gate, B, L, V, walk="maxs
         _ptr(path_score), _ptr(path_q), _ptr(tables), _ptr(target), _ptr(accept_len), _ptr(next_token),
         _ptr(dev_status), _stream(stream)))
     return path_tok, path_slot, path_score, path_q, tables, accept_len, next_token
+
+
+RECORD_WORDS = 36   # one partial record: max, sum, 2 unused, 16 values, 16 indices
+
+
+def dflash_lmhead_topk_records(M: int, V: int, d: int) -> int:
+    return int(lib.dflash_lmhead_topk_records(M, V, d))
+
+
+def dflash_lmhead_topk_partial(H, W, v_offset=0, records=None, dev_status=None, stream=None):
+    """Partial records [M, P, 36] (float32 words) of H . W^T over this shard of
+    the head, vocabulary indices shifted by v_offset."""
+    _need(H, "H", torch.bfloat16)
+    _need(W, "W", torch.bfloat16)
+    M, d = H.shape
+    V = W.shape[0]
+    P = dflash_lmhead_topk_records(M, V, d)
+    if P <= 0:
+        raise DFlashError("dflash_lmhead_topk_records", DFLASH_ERR_INVALID_ARG)
+    records = _out(records, "records", torch.float32, (M, P, RECORD_WORDS), H.device)
+    _check("dflash_lmhead_topk_partial", lib.dflash_lmhead_topk_partial(
+        _ptr(H), _ptr(W), M, V, d, int(v_offset), _ptr(records), records.numel() * 4, _ptr(dev_status),
+        _stream(stream)))
+    return records
+
+
+def dflash_lmhead_topk_merge(records, topk_logp=None, topk_idx=None, lse=None, stream=None):
+    """records [nrank, M, P, 36] float32 -> (topk_logp [M,16], topk_idx [M,16], lse [M])."""
+    _need(records, "records", torch.float32)
+    if records.dim() == 3:
+        records = records.unsqueeze(0)
+    nrank, M, P, w = records.shape
+    if w != RECORD_WORDS:
+        raise ValueError("records must have 36 words per record")
+    topk_logp = _out(topk_logp, "topk_logp", torch.float32, (M, K_TOP), records.device)
+    topk_idx = _out(topk_idx, "topk_idx", torch.int32, (M, K_TOP), records.device)
+    lse = _out(lse, "lse", torch.float32, (M,), records.device)
+    _check("dflash_lmhead_topk_merge", lib.dflash_lmhead_topk_merge(
+        _ptr(records), M, P, nrank, K_TOP, _ptr(topk_logp), _ptr(topk_idx), _ptr(lse), _stream(stream)))
+    return topk_logp, topk_idx, lse

@@ -440,6 +440,58 @@ struct TopState {
     }
   }
 
+  // Keep the 16 best of this list and another sorted list.  The elementwise
+  // better of v[k] and o[15-k] holds exactly those 16 as a bitonic sequence
+  // (one list descending against the other ascending); four half-cleaner
+  // stages sort it.  48 compare-exchanges with static indices, no serial
+  // insertion chain.
+  __device__ __forceinline__ void merge_bitonic(const float (&ov)[KTOP], const int (&oi)[KTOP]) {
+#pragma unroll
+    for (int k = 0; k < KTOP; ++k) {
+      const bool take = better(ov[KTOP - 1 - k], oi[KTOP - 1 - k], v[k], i[k]);
+      v[k] = take ? ov[KTOP - 1 - k] : v[k];
+      i[k] = take ? oi[KTOP - 1 - k] : i[k];
+    }
+#pragma unroll
+    for (int j = KTOP / 2; j >= 1; j >>= 1) {
+#pragma unroll
+      for (int k = 0; k < KTOP; ++k)
+        if ((k & j) == 0) cex(k, k + j, true);
+    }
+  }
+
+  // Make the list the 16 values x[jj] (indices base + jj), sorted by a
+  // bitonic sorting network: the fast way to fill an empty list.
+  __device__ __forceinline__ void assign_sorted16(const float (&x)[KTOP], int base) {
+#pragma unroll
+    for (int k = 0; k < KTOP; ++k) {
+      v[k] = x[k];
+      i[k] = base + k;
+    }
+#pragma unroll
+    for (int size = 2; size <= KTOP; size <<= 1) {
+#pragma unroll
+      for (int stride = size / 2; stride > 0; stride >>= 1) {
+#pragma unroll
+        for (int k = 0; k < KTOP; ++k) {
+          const int partner = k ^ stride;
+          if (partner > k) cex(k, partner, (k & size) == 0);
+        }
+      }
+    }
+  }
+
+  // Compare-exchange entries a < b: desc puts the better one at a.
+  __device__ __forceinline__ void cex(int a, int b, bool desc) {
+    const bool sw = desc ? better(v[b], i[b], v[a], i[a]) : better(v[a], i[a], v[b], i[b]);
+    const float tv = v[a];
+    const int ti = i[a];
+    v[a] = sw ? v[b] : v[a];
+    i[a] = sw ? i[b] : i[a];
+    v[b] = sw ? tv : v[b];
+    i[b] = sw ? ti : i[b];
+  }
+
   // Insert the entries of another sorted list while they beat the 16th entry.
   __device__ __forceinline__ void insert_sorted(const float (&ov)[KTOP], const int (&oi)[KTOP]) {
 #pragma unroll

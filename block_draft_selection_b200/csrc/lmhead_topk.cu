@@ -88,6 +88,7 @@ struct Params {
   int b_widths[4];   // STREAM: the tile widths, one tensor map each
   int merge_halves;  // one run per unit: the two column halves merge in-kernel
   int store_only;    // plain GEMM: write z to z_dbg, no log-softmax / top-16
+  int v_offset;      // added to every vocabulary index written to a record
   // outputs
   Partial* part;     // [M][P]
   int P;
@@ -95,6 +96,14 @@ struct Params {
   int* status;
   unsigned long long timeout_ns;
 };
+
+// A record with the vocabulary indices shifted by `off` (a shard's first row).
+__device__ __forceinline__ void store_record(Partial* dst, const TopState& st, int off) {
+  int gi[KTOP];
+#pragma unroll
+  for (int k = 0; k < KTOP; ++k) gi[k] = st.i[k] == 0x7fffffff ? st.i[k] : st.i[k] + off;
+  store_partial(dst, st.m, st.s, st.v, gi);
+}
 
 struct SmemLayout {
   uint32_t a, b, bars, misc, total;
@@ -404,10 +413,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int row = t.a_row + trow;
       const int nch = t.n_cols / 16;
       const int split = (nch + 1) >> 1;
-      // warps whose 32 rows are all past M only hand the buffer back
+      // the two warps of a lane quarter split the columns; warps whose 32 rows
+      // are all past M only hand the buffer back
+      const int ch_begin = half ? split : 0;
       const int ch_end = t.a_row + quarter * 32 >= p.M ? 0 : (half ? nch : split);
       const uint32_t taddr = tmem_base + static_cast<uint32_t>(tb * TILE_N) + lane_off;
-      for (int ch = half ? split : 0; ch < ch_end; ++ch) {
+      for (int ch = ch_begin; ch < ch_end; ++ch) {
         const int c0 = ch * 16;
         const int vbase = t.v0 + c0;
         if (vbase >= p.V) break;
@@ -442,11 +453,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int jj = 0; jj < 16; ++jj)
           if (jj < nvalid) st.s += __expf(x[jj] - st.m);
         // Candidates of this chunk that can enter the list; each lane then
-        // inserts only its own, so the warp loops max_lane(count) times.
+        // inserts only its own, so the warp loops max_lane(count) times.  An
+        // empty list (a run's first chunk) is filled by sorting the chunk.
         uint32_t pend = 0;
+        if (nvalid == 16 && st.v[0] == -INFINITY) {
+          st.assign_sorted16(x, vbase);
+        } else {
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj)
-          if (jj < nvalid && x[jj] > st.v[KTOP - 1]) pend |= 1u << jj;
+          for (int jj = 0; jj < 16; ++jj)
+            if (jj < nvalid && x[jj] > st.v[KTOP - 1]) pend |= 1u << jj;
+        }
         while (__any_sync(0xffffffffu, pend != 0)) {
           if (pend) {
             const int jj = __ffs(pend) - 1;
@@ -475,7 +491,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           run_slot = t.slot;
           run_row = row;
         } else if (row < p.M)
-          store_partial(p.part + static_cast<size_t>(row) * p.P + 2 * t.slot + half, st.m, st.s, st.v, st.i);
+          store_record(p.part + static_cast<size_t>(row) * p.P + 2 * t.slot + half, st, p.v_offset);
       }
     }
     if (p.merge_halves && !p.store_only) {
@@ -502,8 +518,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           oi[k] = __float_as_int(xs[18 + k]);
         }
         st.merge_lse(xs[0], xs[1]);
-        st.insert_sorted(ov, oi);
-        store_partial(p.part + static_cast<size_t>(run_row) * p.P + run_slot, st.m, st.s, st.v, st.i);
+        st.merge_bitonic(ov, oi);
+        store_record(p.part + static_cast<size_t>(run_row) * p.P + run_slot, st, p.v_offset);
       }
     }
   }
@@ -577,29 +593,6 @@ __device__ __forceinline__ void warp_merge(TopState& st, float& out_v, int& out_
   }
 }
 
-// Fold a lane's share of a row's partial records (q = first, first+step, ...)
-// into its list; records are loaded one ahead so loads overlap the work.
-__device__ __forceinline__ void fold_records(TopState& st, const Partial* base, int first, int step, int P) {
-  if (first >= P) return;
-  PartialRegs cur, nxt;
-  cur.load(base + first);
-  if (first + step < P) nxt.load(base + first + step);
-  // the first record is already a sorted list: it becomes the starting state
-  st.m = cur.m();
-  st.s = cur.s();
-  cur.lists(st.v, st.i);
-  cur = nxt;
-  for (int q = first + step; q < P; q += step) {
-    if (q + step < P) nxt.load(base + q + step);
-    st.merge_lse(cur.m(), cur.s());
-    float rv[KTOP];
-    int ri[KTOP];
-    cur.lists(rv, ri);
-    st.insert_sorted(rv, ri);
-    cur = nxt;
-  }
-}
-
 // Threshold-and-rank merge: one CTA per row, no serial list merging.
 // Every record is a sorted list, so any 16 entries of the row bound its 16th
 // best value from below.  Pass 1 merges the records' (m, s) and takes as that
@@ -616,8 +609,8 @@ __device__ __forceinline__ void fold_records(TopState& st, const Partial* base, 
 // back to folding the records list by list.
 constexpr int MR_CAP = 1024;
 
-template <int NT>
-__global__ void __launch_bounds__(NT) merge_kernel_rank(const Partial* __restrict__ part, int M, int P,
+template <int NT, bool MULTI>
+__global__ void __launch_bounds__(NT) merge_kernel_rank(const Partial* __restrict__ part, int M, int Pr, int nrank,
                                                         float* __restrict__ topk_logp,
                                                         int32_t* __restrict__ topk_idx,
                                                         float* __restrict__ lse) {
@@ -631,7 +624,14 @@ __global__ void __launch_bounds__(NT) merge_kernel_rank(const Partial* __restric
   __shared__ float sh_lse, sh_tau;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int row = blockIdx.x;
-  const Partial* base = part + static_cast<size_t>(row) * P;
+  // records [nrank][M][Pr]: record q of this row is rank q / Pr's record q % Pr
+  const int P = MULTI ? Pr * nrank : Pr;
+  const Partial* base = part + static_cast<size_t>(row) * Pr;
+  auto rec = [&](int q) -> const Partial* {
+    if (!MULTI) return base + q;
+    const int rk = q / Pr;
+    return part + (static_cast<size_t>(rk) * M + row) * Pr + (q - rk * Pr);
+  };
   pdl_wait();
   pdl_trigger();
   if (tid == 0) {
@@ -647,7 +647,7 @@ __global__ void __launch_bounds__(NT) merge_kernel_rank(const Partial* __restric
   st.s = 0.f;
   float tau16 = -INFINITY;
   for (int q = tid; q < P; q += NT) {
-    const float* r = reinterpret_cast<const float*>(base + q);
+    const float* r = reinterpret_cast<const float*>(rec(q));
     const float4 h = __ldg(reinterpret_cast<const float4*>(r));
     st.merge_lse(h.x, h.y);
     tau16 = fmaxf(tau16, __ldg(r + 4 + (KTOP - 1)));
@@ -696,7 +696,7 @@ __global__ void __launch_bounds__(NT) merge_kernel_rank(const Partial* __restric
 
   // pass 2: gather the entries >= tau (a prefix of each record)
   for (int q = tid; q < P; q += NT) {
-    const float4* r = reinterpret_cast<const float4*>(base + q);
+    const float4* r = reinterpret_cast<const float4*>(rec(q));
     float v[KTOP];
     int ix[KTOP];
 #pragma unroll
@@ -745,7 +745,15 @@ __global__ void __launch_bounds__(NT) merge_kernel_rank(const Partial* __restric
     // ties overflowed a buffer: fold the records list by list
     TopState fs;
     fs.reset();
-    fold_records(fs, base, tid, NT, P);
+    for (int q = tid; q < P; q += NT) {
+      PartialRegs r;
+      r.load(rec(q));
+      fs.merge_lse(r.m(), r.s());
+      float rv[KTOP];
+      int ri[KTOP];
+      r.lists(rv, ri);
+      fs.merge_bitonic(rv, ri);
+    }
     float v;
     int ix;
     warp_merge(fs, v, ix);
@@ -986,9 +994,26 @@ static cudaError_t launch_main(const Plan& pl, const CUtensorMap& ta, const CUte
                                PAIR ? 2 : 1, ta, tb[0], tb[1], tb[2], tb[3], pl.p);
 }
 
+static cudaError_t launch_merge(const Partial* part, int M, int Pr, int nrank, float* topk_logp,
+                                int32_t* topk_idx, float* lse, cudaStream_t st) {
+  const bool wide = static_cast<long long>(Pr) * nrank > 128;
+  if (nrank == 1)
+    return wide ? launch_kernel(merge_kernel_rank<256, false>, dim3(M), dim3(256), 0, st, part, M, Pr, 1, topk_logp,
+                                topk_idx, lse)
+                : launch_kernel(merge_kernel_rank<128, false>, dim3(M), dim3(128), 0, st, part, M, Pr, 1, topk_logp,
+                                topk_idx, lse);
+  return wide ? launch_kernel(merge_kernel_rank<256, true>, dim3(M), dim3(256), 0, st, part, M, Pr, nrank, topk_logp,
+                              topk_idx, lse)
+              : launch_kernel(merge_kernel_rank<128, true>, dim3(M), dim3(128), 0, st, part, M, Pr, nrank, topk_logp,
+                              topk_idx, lse);
+}
+
+// records_only: run the GEMM + epilogue kernel alone (the records stay in ws
+// for a later merge, e.g. after gathering every shard's records); v_offset is
+// added to the records' vocabulary indices.
 static int launch(const dflash_bf16* H, const dflash_bf16* W, int M, int V, int d, float* topk_logp,
                   int32_t* topk_idx, float* lse, float* z_dbg, void* ws, size_t ws_bytes, int* dev_status,
-                  void* stream, bool store_only = false) {
+                  void* stream, bool store_only = false, bool records_only = false, int v_offset = 0) {
   if (!H || !W || (!ws && !store_only)) return DFLASH_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(H) & 15) || (reinterpret_cast<uintptr_t>(W) & 15) ||
       (reinterpret_cast<uintptr_t>(ws) & 255) || (store_only && (reinterpret_cast<uintptr_t>(z_dbg) & 15)))
@@ -999,6 +1024,7 @@ static int launch(const dflash_bf16* H, const dflash_bf16* W, int M, int V, int 
   Params& p = pl.p;
   p.part = static_cast<Partial*>(ws);
   p.store_only = store_only ? 1 : 0;
+  p.v_offset = v_offset;
   p.z_dbg = z_dbg;
   p.status = dev_status;
   p.timeout_ns = timeout_ns_from_env();
@@ -1022,15 +1048,8 @@ static int launch(const dflash_bf16* H, const dflash_bf16* W, int M, int V, int 
   else
     e = pl.pair ? launch_main<MODE_LARGE, true>(pl, ta, tb, st) : launch_main<MODE_LARGE, false>(pl, ta, tb, st);
   if (e != cudaSuccess) return DFLASH_ERR_CUDA;
-  if (z_dbg == nullptr && !store_only) {
-    const Partial* part = p.part;
-    cudaError_t me;
-    if (p.P > 128) {
-      me = launch_kernel(merge_kernel_rank<256>, dim3(M), dim3(256), 0, st, part, M, p.P, topk_logp, topk_idx, lse);
-    } else {
-      me = launch_kernel(merge_kernel_rank<128>, dim3(M), dim3(128), 0, st, part, M, p.P, topk_logp, topk_idx, lse);
-    }
-    if (me != cudaSuccess) return DFLASH_ERR_CUDA;
+  if (z_dbg == nullptr && !store_only && !records_only) {
+    if (launch_merge(p.part, M, p.P, 1, topk_logp, topk_idx, lse, st) != cudaSuccess) return DFLASH_ERR_CUDA;
   }
   return DFLASH_OK;
 }
@@ -1061,6 +1080,30 @@ extern "C" int dflash_gemm_bf16(const dflash_bf16* A, const dflash_bf16* B, floa
                                 void* stream) {
   if (!C || N < 16) return DFLASH_ERR_INVALID_ARG;
   return dflash::lm::launch(A, B, M, N, K, nullptr, nullptr, nullptr, C, nullptr, 0, nullptr, stream, true);
+}
+
+extern "C" int dflash_lmhead_topk_records(int M, int V, int d) {
+  dflash::lm::Plan pl;
+  if (!dflash::lm::make_plan(M, V, d, dflash::lm::num_sms_current(), pl)) return 0;
+  return pl.p.P;
+}
+
+extern "C" int dflash_lmhead_topk_partial(const dflash_bf16* H, const dflash_bf16* W, int M, int V, int d,
+                                          int v_offset, void* records, size_t records_bytes, int* dev_status,
+                                          void* stream) {
+  if (!records || v_offset < 0) return DFLASH_ERR_INVALID_ARG;
+  return dflash::lm::launch(H, W, M, V, d, nullptr, nullptr, nullptr, nullptr, records, records_bytes, dev_status,
+                            stream, false, true, v_offset);
+}
+
+extern "C" int dflash_lmhead_topk_merge(const void* records, int M, int P, int nrank, int K, float* topk_logp,
+                                        int32_t* topk_idx, float* lse, void* stream) {
+  if (!records || !topk_logp || !topk_idx || K != dflash::KTOP || M < 1 || P < 1 || nrank < 1)
+    return DFLASH_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(records) & 15) return DFLASH_ERR_INVALID_ARG;
+  const cudaError_t e = dflash::lm::launch_merge(static_cast<const dflash::Partial*>(records), M, P, nrank, topk_logp,
+                                                 topk_idx, lse, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------------------

@@ -211,6 +211,34 @@ int dflash_select_verify(const float* topk_logp, const int32_t* topk_idx, const 
                          int32_t* next_token, int* dev_status, void* stream);
 
 /*
+ * Vocabulary-parallel LM head: each rank owns rows [v_offset, v_offset + V)
+ * of the full head and produces per-row partial records; the records of all
+ * ranks, gathered in rank order, merge into the full vocabulary's top-16.
+ * Same definition as dflash_lmhead_topk over the concatenated head.
+ *
+ * dflash_lmhead_topk_records(M, V, d): records per row P that a call with
+ * this shard shape writes (0 if unsupported).  Every rank of one gather must
+ * use the same P: pad a shorter rank's buffer with empty records (m = -inf,
+ * s = 0, values -inf, indices 0x7fffffff), which the merge ignores.
+ *
+ * dflash_lmhead_topk_partial: the GEMM + online log-sum-exp + top-16 kernel
+ * alone over W [V, d] (this rank's shard); writes records [M][P] into
+ * `records` (dflash_lmhead_topk_workspace(M, V, d) bytes, 256-byte aligned)
+ * with every vocabulary index shifted by v_offset >= 0.  A record is 36
+ * 32-bit words: running max, sum of exp(z - max), 2 unused, the 16 best
+ * values (descending), their 16 indices (int32 bits).
+ *
+ * dflash_lmhead_topk_merge: records [nrank][M][P] (16-byte aligned) ->
+ * topk_logp, topk_idx [M, 16], lse [M] (nullable), exactly as
+ * dflash_lmhead_topk's own merge.  K must be 16.
+ */
+int dflash_lmhead_topk_records(int M, int V, int d);
+int dflash_lmhead_topk_partial(const dflash_bf16* H, const dflash_bf16* W, int M, int V, int d, int v_offset,
+                               void* records, size_t records_bytes, int* dev_status, void* stream);
+int dflash_lmhead_topk_merge(const void* records, int M, int P, int nrank, int K, float* topk_logp,
+                             int32_t* topk_idx, float* lse, void* stream);
+
+/*
  * Walk from the last verified token.
  * "DFlash 2: Keep Drafting Parallel", section "a lightweight path selector":
  * starting from the last verified token, the walk over the precomputed pair

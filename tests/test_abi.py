@@ -72,6 +72,7 @@ def test_host_side_rejections(lib):
     assert lib.dflash_path_walk(fake, fake, fake, fake, fake, None, 1.0, 1, 4, 16, 32, 100,
                                 fake, None, None, None, fake, None, None, None, None) == 1
     # rejection verify: temperature <= 0, L > 31, V too large, workspace too small
+    i32 = ctypes.c_int
     lib.dflash_verify_rejection.argtypes = ([vp, f32] + [vp] * 6 + [ctypes.c_int] * 3 + [vp, vp, vp,
                                             ctypes.c_size_t, vp, vp])
     big = ctypes.c_size_t(1 << 30)
@@ -83,6 +84,13 @@ def test_host_side_rejections(lib):
     assert lib.dflash_verify_rejection(*args(1.0, 1, 4, 1000, ctypes.c_size_t(8))) == 4
     lib.dflash_verify_rejection_workspace.restype = ctypes.c_size_t
     assert lib.dflash_verify_rejection_workspace(2, 3, 8193) == 2 * 4 * 2 * 16
+    # vocabulary-parallel pieces: negative offset, K != 16, bad record counts
+    lib.dflash_lmhead_topk_partial.argtypes = [vp, vp, i32, i32, i32, i32, vp, ctypes.c_size_t, vp, vp]
+    assert lib.dflash_lmhead_topk_partial(fake, fake, 4, 4096, 256, -16, fake, big, None, None) == 1
+    lib.dflash_lmhead_topk_merge.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp]
+    assert lib.dflash_lmhead_topk_merge(fake, 4, 148, 2, 15, fake, fake, None, None) == 1
+    assert lib.dflash_lmhead_topk_merge(fake, 4, 0, 2, 16, fake, fake, None, None) == 1
+    assert lib.dflash_lmhead_topk_merge(fake, 4, 148, 0, 16, fake, fake, None, None) == 1
     # context-gated scorer: e not a multiple of 8, L > 16, K != 16, unknown walk, sampling without uniforms
     i32 = ctypes.c_int
     lib.dflash_ctx_project.argtypes = [vp] * 6 + [i32] * 5 + [vp, vp, vp, ctypes.c_size_t, vp, vp]

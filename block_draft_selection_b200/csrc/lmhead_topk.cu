@@ -593,6 +593,29 @@ __device__ __forceinline__ void warp_merge(TopState& st, float& out_v, int& out_
   }
 }
 
+// Fold a lane's share of a row's partial records (q = first, first+step, ...)
+// into its list; records are loaded one ahead so loads overlap the work.
+__device__ __forceinline__ void fold_records(TopState& st, const Partial* base, int first, int step, int P) {
+  if (first >= P) return;
+  PartialRegs cur, nxt;
+  cur.load(base + first);
+  if (first + step < P) nxt.load(base + first + step);
+  // the first record is already a sorted list: it becomes the starting state
+  st.m = cur.m();
+  st.s = cur.s();
+  cur.lists(st.v, st.i);
+  cur = nxt;
+  for (int q = first + step; q < P; q += step) {
+    if (q + step < P) nxt.load(base + q + step);
+    st.merge_lse(cur.m(), cur.s());
+    float rv[KTOP];
+    int ri[KTOP];
+    cur.lists(rv, ri);
+    st.insert_sorted(rv, ri);
+    cur = nxt;
+  }
+}
+
 // Threshold-and-rank merge: one CTA per row, no serial list merging.
 // Every record is a sorted list, so any 16 entries of the row bound its 16th
 // best value from below.  Pass 1 merges the records' (m, s) and takes as that
@@ -745,14 +768,18 @@ __global__ void __launch_bounds__(NT) merge_kernel_rank(const Partial* __restric
     // ties overflowed a buffer: fold the records list by list
     TopState fs;
     fs.reset();
-    for (int q = tid; q < P; q += NT) {
-      PartialRegs r;
-      r.load(rec(q));
-      fs.merge_lse(r.m(), r.s());
-      float rv[KTOP];
-      int ri[KTOP];
-      r.lists(rv, ri);
-      fs.merge_bitonic(rv, ri);
+    if (MULTI) {
+      for (int q = tid; q < P; q += NT) {
+        PartialRegs r;
+        r.load(rec(q));
+        fs.merge_lse(r.m(), r.s());
+        float rv[KTOP];
+        int ri[KTOP];
+        r.lists(rv, ri);
+        fs.merge_bitonic(rv, ri);
+      }
+    } else {
+      fold_records(fs, base, tid, NT, P);
     }
     float v;
     int ix;

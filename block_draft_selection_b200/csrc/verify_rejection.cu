@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(T1) row_stats_kernel(const float* __restrict__
     for (int j = 0; j < EPT1 / 4; ++j) {
       const int v = v0 + (j * T1 + tid) * 4;
       float4 t = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-      if (v < V) t = __ldcs(reinterpret_cast<const float4*>(zr + v));  // V % 4 == 0: all four in range
+      if (v < V) t = __ldg(reinterpret_cast<const float4*>(zr + v));  // V % 4 == 0: all four in range
       x[4 * j + 0] = t.x;
       x[4 * j + 1] = t.y;
       x[4 * j + 2] = t.z;
@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(T1) row_stats_kernel(const float* __restrict__
 #pragma unroll
     for (int j = 0; j < EPT1; ++j) {
       const int v = v0 + j * T1 + tid;
-      x[j] = v < V ? __ldcs(zr + v) : -INFINITY;
+      x[j] = v < V ? __ldg(zr + v) : -INFINITY;
     }
   }
   float xm = -INFINITY;
@@ -134,6 +134,9 @@ __global__ void __launch_bounds__(T2) reject_kernel(
   __shared__ double wsum[T2 / 32];
   __shared__ int sh_n, sh_slice, sh_pick, sh_before, sh_last;
   __shared__ double sh_excl, sh_target;
+  __shared__ int pc_idx[MAX_L][KC];    // every position's candidates, their q and logits,
+  __shared__ float pc_q[MAX_L][KC];    // read up front (the rejected position is not yet
+  __shared__ float pc_z[MAX_L][KC];    // known, and these loads need not wait for it)
 
   pdl_wait();
   pdl_trigger();
@@ -144,6 +147,40 @@ __global__ void __launch_bounds__(T2) reject_kernel(
     sh_pick = INT_MAX;
     sh_before = -1;
     sh_last = -1;
+  }
+  // warp 0, lane i < L: drafted position i's token, slot, q and target logit
+  int dx = 0;
+  double dq = 0.0, du = 0.0;
+  float dz = 0.f;
+  if (warp == 0 && lane < L) {
+    const size_t di = static_cast<size_t>(b) * L + lane;
+    dx = draft[di];
+    int sl = draft_slot[di];
+    if (dx < 0 || dx >= V || sl < 0 || sl >= KC) {
+      set_status(status, DFLASH_ERR_BAD_INDEX);
+      dx = min(max(dx, 0), V - 1);
+      sl = min(max(sl, 0), KC - 1);
+    }
+    dq = draft_q[di * KC + sl];
+    du = u_accept[di];
+    dz = z[(row0 + lane) * V + dx];
+  }
+  // threads 32 .. 32 + 16 L - 1: candidate k of position i
+  if (tid >= 32 && tid < 32 + KC * L) {
+    const int i = (tid - 32) / KC;
+    const int k = (tid - 32) - i * KC;
+    const size_t ci = (static_cast<size_t>(b) * L + i) * KC + k;
+    int v = cand_idx[ci];
+    float zv = 0.f;
+    if (v < 0 || v >= V) {
+      set_status(status, DFLASH_ERR_BAD_INDEX);
+      v = -1;
+    } else {
+      zv = z[(row0 + i) * V + v];
+    }
+    pc_idx[i][k] = v;
+    pc_q[i][k] = draft_q[ci];
+    pc_z[i][k] = zv;
   }
 
   // A. each row's max and sum from its slices (warp i -> row i)
@@ -167,21 +204,12 @@ __global__ void __launch_bounds__(T2) reject_kernel(
   }
   __syncthreads();
 
-  // B. acceptance tests, lane i for drafted position i
+  // B. acceptance tests, lane i for drafted position i (values read above)
   if (warp == 0) {
     bool reject = false;
     if (lane < L) {
-      const size_t di = static_cast<size_t>(b) * L + lane;
-      int x = draft[di];
-      int sl = draft_slot[di];
-      if (x < 0 || x >= V || sl < 0 || sl >= KC) {
-        set_status(status, DFLASH_ERR_BAD_INDEX);
-        x = min(max(x, 0), V - 1);
-        sl = min(max(sl, 0), KC - 1);
-      }
-      const double q = draft_q[di * KC + sl];
-      const double p = exp2(static_cast<double>(z[(row0 + lane) * V + x]) * c - row_m[lane]) / row_s[lane];
-      reject = !(static_cast<double>(u_accept[di]) * q <= p);
+      const double p = exp2(static_cast<double>(dz) * c - row_m[lane]) / row_s[lane];
+      reject = !(du * dq <= p);
     }
     const unsigned mask = __ballot_sync(FULL, reject);
     const int n = mask ? __ffs(mask) - 1 : L;
@@ -199,19 +227,8 @@ __global__ void __launch_bounds__(T2) reject_kernel(
 
   // C. slice masses of p_R, minus q_n at the candidates (rejection only)
   if (tid < KC) {
-    int v = -1;
-    float q = 0.f;
-    if (n < L) {
-      const size_t ci = (static_cast<size_t>(b) * L + n) * KC + tid;
-      v = cand_idx[ci];
-      q = draft_q[ci];
-      if (v < 0 || v >= V) {
-        set_status(status, DFLASH_ERR_BAD_INDEX);
-        v = -1;
-      }
-    }
-    cand_s[tid] = v;
-    q_s[tid] = q;
+    cand_s[tid] = n < L ? pc_idx[n][tid] : -1;
+    q_s[tid] = n < L ? pc_q[n][tid] : 0.f;
   }
   for (int j = tid; j < S; j += T2) {
     const Part p = part[R * S + j];
@@ -220,7 +237,7 @@ __global__ void __launch_bounds__(T2) reject_kernel(
   __syncthreads();
   if (tid < KC && cand_s[tid] >= 0) {
     const int v = cand_s[tid];
-    const double pv = exp2(static_cast<double>(zr[v]) * c - mx) / sR;
+    const double pv = exp2(static_cast<double>(pc_z[n][tid]) * c - mx) / sR;
     atomicAdd(&mass[v / SPAN], fmax(0.0, pv - static_cast<double>(q_s[tid])) - pv);
   }
   __syncthreads();

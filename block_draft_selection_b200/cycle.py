@@ -6,12 +6,39 @@ verification -- on buffers owned by the object.  `run()` copies one step's
 inputs from pinned host buffers to the device, runs the cycle and copies its
 results back, all captured once into a CUDA graph so a step costs one graph
 launch on the host.  Weights (W, E, M, conv taps) stay on the device.
+
+The step's inputs live in one pinned host arena and one device arena with the
+same layout (each tensor at a 256-byte-aligned offset), and so do its results:
+a step moves its inputs with one host-to-device copy and its results with one
+device-to-host copy.
 """
 from __future__ import annotations
 
 import torch
 
 from . import _binding as b
+
+
+def _arena(specs, device, pinned=False, align=256):
+    """One byte buffer holding tensors of the given (name, shape, dtype) at
+    aligned offsets; returns (buffer, {name: view})."""
+    offs, off = {}, 0
+    for name, shape, dt in specs:
+        off = (off + align - 1) // align * align
+        n = 1
+        for x in shape:
+            n *= x
+        offs[name] = (off, shape, dt)
+        off += n * torch.tensor([], dtype=dt).element_size()
+    buf = torch.empty(max(off, 1), dtype=torch.uint8, device=device, pin_memory=pinned)
+    views = {}
+    for name, (o, shape, dt) in offs.items():
+        n = 1
+        for x in shape:
+            n *= x
+        nb = n * torch.tensor([], dtype=dt).element_size()
+        views[name] = buf[o:o + nb].view(dt).view(shape)
+    return buf, views
 
 
 class DraftCycle:
@@ -22,20 +49,21 @@ class DraftCycle:
         V, d = W.shape
         M = B * L
         e = lambda shape, dt: torch.empty(shape, dtype=dt, device=dev)
-        # device buffers
-        self.H, self.x, self.prev = e((M, d), torch.bfloat16), e((B, P, d), torch.bfloat16), e((B, d), torch.bfloat16)
-        self.target = e((B, L + 1), torch.int32)
-        self.y = e((B, P, d), torch.bfloat16)
+        ins = [("H", (M, d), torch.bfloat16), ("x", (B, P, d), torch.bfloat16), ("prev", (B, d), torch.bfloat16),
+               ("target", (B, L + 1), torch.int32)]
+        outs = [("path_tok", (B, L), torch.int32), ("accept_len", (B,), torch.int32),
+                ("next_token", (B,), torch.int32), ("y", (B, P, d), torch.bfloat16)]
+        # device arenas (inputs, results) and their pinned host twins
+        self._din, din = _arena(ins, dev)
+        self._dout, dout = _arena(outs, dev)
+        self._hin, self.host_in = _arena(ins, "cpu", pinned=True)
+        self._hout, self.host_out = _arena(outs, "cpu", pinned=True)
+        self.H, self.x, self.prev, self.target = din["H"], din["x"], din["prev"], din["target"]
+        self.tok, self.acc, self.nxt, self.y = dout["path_tok"], dout["accept_len"], dout["next_token"], dout["y"]
         self.lp, self.ix, self.lse = e((M, 16), torch.float32), e((M, 16), torch.int32), e((M,), torch.float32)
-        self.tok, self.slot = e((B, L), torch.int32), e((B, L), torch.int32)
-        self.score, self.acc, self.nxt = e((B,), torch.float32), e((B,), torch.int32), e((B,), torch.int32)
+        self.slot, self.score = e((B, L), torch.int32), e((B,), torch.float32)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.ws = b.workspace(M, V, d, dev)
-        # pinned host buffers: inputs the caller fills, results the cycle returns
-        pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-        self.host_in = {"H": pin(self.H), "x": pin(self.x), "prev": pin(self.prev), "target": pin(self.target)}
-        self.host_out = {"path_tok": pin(self.tok), "accept_len": pin(self.acc), "next_token": pin(self.nxt),
-                         "y": pin(self.y)}
         self._graph = None
         if use_graph:
             self._capture()
@@ -50,12 +78,9 @@ class DraftCycle:
                                accept_len=self.acc, next_token=self.nxt, dev_status=self.status)
 
     def _step(self):
-        for name, dst in (("H", self.H), ("x", self.x), ("prev", self.prev), ("target", self.target)):
-            dst.copy_(self.host_in[name], non_blocking=True)
+        self._din.copy_(self._hin, non_blocking=True)      # one host-to-device copy
         self.kernels()
-        for name, src in (("path_tok", self.tok), ("accept_len", self.acc), ("next_token", self.nxt),
-                          ("y", self.y)):
-            self.host_out[name].copy_(src, non_blocking=True)
+        self._hout.copy_(self._dout, non_blocking=True)    # one device-to-host copy
 
     def _capture(self):
         side = torch.cuda.Stream()
@@ -78,5 +103,6 @@ class DraftCycle:
         return self.host_out
 
     def io_bytes(self):
-        nb = lambda d: int(sum(t.numel() * t.element_size() for t in d.values()))
-        return nb(self.host_in), nb(self.host_out)
+        """Bytes a step copies host-to-device and device-to-host (the arenas,
+        alignment padding included)."""
+        return int(self._hin.numel()), int(self._hout.numel())

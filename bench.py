@@ -199,7 +199,7 @@ class Step:
 
     TEMPERATURE = 1.0
 
-    def __init__(self, w: syn.Workload, rank: int, device, cycle: str = "greedy"):
+    def __init__(self, w: syn.Workload, rank: int, device, cycle: str = "greedy", conv: str = "static"):
         import torch
         import block_draft_selection_b200 as bds
         self.bds, self.torch, self.w = bds, torch, w
@@ -226,7 +226,20 @@ class Step:
         self.tok, self.slot = e((w.B, w.L), torch.int32), e((w.B, w.L), torch.int32)
         self.score, self.acc, self.nxt = e(w.B, torch.float32), e(w.B, torch.int32), e(w.B, torch.int32)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
-        self.cycle = cycle
+        self.cycle, self.conv = cycle, conv
+        if conv == "dynamic":
+            self.Wc = bds.bf16_tensor(syn.conv_correction(w), dev)
+            self.cws = torch.empty(max(1, int(bds.lib.dflash_conv2tap_dynamic_workspace(w.B, w.P, w.d))),
+                                   dtype=torch.uint8, device=dev)
+        if cycle == "ctx":
+            # the pages' context-gated scorer: tied embeddings (the head), e = 256
+            Pab, Pg = syn.ctx_scorer_weights(w, 256)
+            self.Pab, self.Pg = bds.bf16_tensor(Pab, dev), bds.bf16_tensor(Pg, dev)
+            self.anchor = torch.from_numpy(syn.anchors(w.B, w.V, wr.seed)).to(dev)
+            self.proj = e((w.B * (1 + 16 * w.L), 512), torch.float32)
+            self.gate = e((w.M, 256), torch.float32)
+            self.pws = torch.empty(max(16, bds.dflash_ctx_project_workspace(w.B, w.L, w.d)), dtype=torch.uint8,
+                                   device=dev)
         if cycle == "sample":
             # the target's logits at the L drafted positions and the bonus
             # position (the library's plain GEMM on the noised hidden states)
@@ -248,9 +261,13 @@ class Step:
     TIMED = STAGES + ("event_pair", "lmhead_select")
     # sample cycle: conv, LM head (2), walk, rejection verification (2)
     LAUNCHES_PER_STEP_SAMPLE = 6
+    # ctx cycle: conv, LM head (2), projections (gather + 2 GEMMs), scores + walk
+    LAUNCHES_PER_STEP_CTX = 7
 
     def launches(self):
-        return self.LAUNCHES_PER_STEP_SAMPLE if self.cycle == "sample" else self.LAUNCHES_PER_STEP
+        n = {"sample": self.LAUNCHES_PER_STEP_SAMPLE, "ctx": self.LAUNCHES_PER_STEP_CTX}.get(
+            self.cycle, self.LAUNCHES_PER_STEP)
+        return n + (1 if self.conv == "dynamic" else 0)   # the dynamic conv adds its correction GEMM
 
     def run(self, marks=None):
         """One cycle.  `marks`: optional {stage name: (event, event)} recorded
@@ -267,7 +284,11 @@ class Step:
                 ev[1].record()
 
         stage("event_pair", lambda: None)    # calibration: two event nodes, nothing between
-        stage("conv2tap", lambda: bds.dflash_conv2tap(self.x, self.a0, self.a1, self.prev, y=self.y))
+        if self.conv == "dynamic":
+            stage("conv2tap", lambda: bds.dflash_conv2tap_dynamic(self.x, self.a0, self.a1, self.Wc, self.prev,
+                                                                  y=self.y, ws=self.cws))
+        else:
+            stage("conv2tap", lambda: bds.dflash_conv2tap(self.x, self.a0, self.a1, self.prev, y=self.y))
         span = marks.get("lmhead_select")
         if span:
             span[0].record()
@@ -283,6 +304,15 @@ class Step:
                                             self.u_acc, self.u_res, accept_len=self.acc, next_token=self.nxt,
                                             ws=self.rws, dev_status=self.status)
             stage("select_verify", walk_verify)
+        elif self.cycle == "ctx":
+            def ctx_select_verify():
+                bds.dflash_ctx_project(self.W, self.H, self.Pab, self.Pg, self.ix, self.anchor, self.w.B, self.w.L,
+                                       proj=self.proj, gate=self.gate, ws=self.pws, dev_status=self.status)
+                bds.dflash_ctx_walk(self.lp, self.ix, self.anchor, self.proj, self.gate, self.w.B, self.w.L,
+                                    self.w.V, walk="maxsum", target=self.target, path_tok=self.tok,
+                                    path_slot=self.slot, path_score=self.score, accept_len=self.acc,
+                                    next_token=self.nxt, dev_status=self.status)
+            stage("select_verify", ctx_select_verify)
         else:
             stage("select_verify", lambda: bds.dflash_select_verify(
                 self.lp, self.ix, self.E, self.Msel, self.target, self.w.B, self.w.L, path_tok=self.tok,
@@ -335,7 +365,7 @@ def gpu_arm(args, w: syn.Workload):
                                 device_id=torch.device("cuda", local_rank))
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
-    step = Step(w, rank, device, args.cycle)
+    step = Step(w, rank, device, args.cycle, args.conv)
 
     def barrier():
         torch.cuda.synchronize()
@@ -397,7 +427,7 @@ def gpu_arm(args, w: syn.Workload):
     # copies the step's inputs from pinned host memory, runs the cycle and
     # copies the results back; the host waits for them every step
     e2e = None
-    if args.cycle == "greedy":
+    if args.cycle == "greedy" and args.conv == "static":
         cyc = bds.DraftCycle(step.W, step.E, step.Msel, step.a0, step.a1, w.B, w.L, w.P)
         cyc.host_in["H"].copy_(step.H)
         cyc.host_in["x"].copy_(step.x)
@@ -423,7 +453,7 @@ def gpu_arm(args, w: syn.Workload):
                "path": "DraftCycle.run(): pinned H2D + conv + LM head + select/verify + D2H, host sync"}
     else:
         e2e = {"value": None, "unit": UNIT, "h2d_bytes_per_step": None, "d2h_bytes_per_step": None,
-               "path": "not measured for the sampled cycle: its target logits live on the device"}
+               "path": "measured for the greedy cycle with static taps only (the metric's path)"}
 
     peaks, peaks_kind = load_peaks()
     alg_bytes, alg_flops = lmhead_algorithmic(w)
@@ -456,10 +486,12 @@ def gpu_arm(args, w: syn.Workload):
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded block_draft_synth; random-init weights of the workload's shapes)",
-            "config": {"workload": w.name if args.cycle == "greedy" else f"{w.name}+sampled-walk(T=1)",
+            "config": {"workload": w.name + {"greedy": "", "sample": "+sampled-walk(T=1)",
+                                              "ctx": "+context-gated-scorer"}[args.cycle]
+                                   + ("+dynamic-conv" if args.conv == "dynamic" else ""),
                        "blocks_per_gpu": w.B, "L": w.L, "M": w.M, "d": w.d, "V": w.V,
                        "K": 16, "r": w.r, "conv": [w.B, w.P, w.d], "parallelism": f"dp{world} (blocks)",
-                       "cycle": args.cycle,
+                       "cycle": args.cycle, "conv": args.conv,
                        "launch": "eager" if args.eager else f"cuda graphs of {chunk} cycles, PDL between kernels",
                        "l2": "inputs larger than L2 (W is %.0f MB > 126 MB)" % (2 * w.V * w.d / 1e6)},
             "e2e": e2e,
@@ -603,9 +635,13 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch each cycle eagerly instead of a CUDA graph")
-    ap.add_argument("--cycle", default="greedy", choices=["greedy", "sample"],
+    ap.add_argument("--cycle", default="greedy", choices=["greedy", "sample", "ctx"],
                     help="greedy: max-sum selection + greedy verification (the metric's path); sample: "
-                         "sampled walk from the last verified token + rejection-sampling verification")
+                         "sampled walk from the last verified token + rejection-sampling verification; ctx: "
+                         "the pages' context-gated scorer, max-sum from the last verified token + greedy "
+                         "verification")
+    ap.add_argument("--conv", default="static", choices=["static", "dynamic"],
+                    help="static base taps (the metric's path) or taps with the per-16-channel correction")
     ap.add_argument("--ref-budget-s", type=float, default=120.0,
                     help="host seconds the --impl reference run aims to take")
     args = ap.parse_args(argv)

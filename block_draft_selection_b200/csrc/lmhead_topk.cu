@@ -89,6 +89,8 @@ struct Params {
   int merge_halves;  // one run per unit: the two column halves merge in-kernel
   int store_only;    // plain GEMM: write z to z_dbg, no log-softmax / top-16
   int v_offset;      // added to every vocabulary index written to a record
+  int ksplit;        // plain GEMM, STREAM: CTAs per tile range, each over 1/ksplit of K
+                     // (partial sums added into z_dbg, which the host zeroes first)
   // outputs
   Partial* part;     // [M][P]
   int P;
@@ -146,7 +148,7 @@ __device__ __forceinline__ bool get_tile(const Params& p, int k, uint32_t rank, 
     // The range is cut into the fewest tiles of at most 256 rows, all of
     // (nearly) equal width: every tile costs a full K loop of MMAs whatever
     // its width, so no CTA carries a sliver tile.
-    const long long G = gridDim.x, c = blockIdx.x;
+    const long long G = gridDim.x / p.ksplit, c = blockIdx.x % G;
     const int u0 = static_cast<int>((c * p.units) / G);
     const int u1 = static_cast<int>(((c + 1) * p.units) / G);
     const int nt = (u1 - u0 + TILE_N / 16 - 1) / (TILE_N / 16);
@@ -266,6 +268,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // Set-up above overlaps the previous kernel; global memory only from here.
   pdl_wait();
   const uint64_t deadline = globaltimer_ns() + p.timeout_ns;
+  // this CTA's share of K (split only for the plain GEMM in STREAM mode)
+  const int ks = MODE == MODE_STREAM ? static_cast<int>(blockIdx.x / (gridDim.x / p.ksplit)) : 0;
+  const int kc0 = ks * p.num_kc / p.ksplit;
+  const int kc1 = (ks + 1) * p.num_kc / p.ksplit;
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
@@ -290,7 +296,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // bytes landing on the leader's barrier per stage (both CTAs of a pair)
         const int b_rows_here = MODE == MODE_STREAM ? t.n_cols : p.b_rows;
         const uint32_t tx = static_cast<uint32_t>((PAIR ? 2 : 1) * (p.a_box + b_rows_here) * BK * 2);
-        for (int kc = 0; kc < p.num_kc; ++kc) {
+        for (int kc = kc0; kc < kc1; ++kc) {
           if (!mbar_wait(empty_bar(s), ph ^ 1u, deadline, abort_flag, p.status)) {
             ok = false;
             break;
@@ -356,7 +362,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(tb * TILE_N);
-        for (int kc = 0; kc < p.num_kc; ++kc) {
+        for (int kc = kc0; kc < kc1; ++kc) {
           if (!mbar_wait(full_bar(s), ph, deadline, abort_flag, p.status)) {
             ok = false;
             break;
@@ -367,7 +373,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / UMMA_K; ++kk) {
             // advance the start address by kk * 32 bytes (encoded >> 4)
-            const uint32_t acc = (kc | kk) != 0 ? 1u : 0u;
+            const uint32_t acc = ((kc - kc0) | kk) != 0 ? 1u : 0u;
             if (PAIR)
               umma_bf16_pair(d_tmem, adesc + 2ull * kk, bdesc + 2ull * kk, idesc, acc);
             else
@@ -427,7 +433,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_ld_wait();
         const int nvalid = min(16, p.V - vbase);
         if (p.store_only) {
-          if (row < p.M) {
+          if (row < p.M && p.ksplit > 1) {
+            float* zr = p.z_dbg + static_cast<size_t>(row) * p.V + vbase;
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj)
+              if (jj < nvalid) atomicAdd(zr + jj, x[jj]);
+          } else if (row < p.M) {
             float* zr = p.z_dbg + static_cast<size_t>(row) * p.V + vbase;
             if (nvalid == 16 && (p.V & 3) == 0) {
 #pragma unroll
@@ -922,6 +933,7 @@ static bool make_plan(int M, int V, int d, int sms, Plan& pl) {
   p.d = d;
   p.num_kc = (d + BK - 1) / BK;
   p.tmem_cols = 2 * TILE_N;
+  p.ksplit = 1;
   if (M <= A_ROWS) {
     pl.mode = MODE_STREAM;
     pl.pair = false;
@@ -1052,6 +1064,19 @@ static int launch(const dflash_bf16* H, const dflash_bf16* W, int M, int V, int 
   p.part = static_cast<Partial*>(ws);
   p.store_only = store_only ? 1 : 0;
   p.v_offset = v_offset;
+  if (store_only && pl.mode == MODE_STREAM) {
+    // few tile ranges and a long K: split K over otherwise idle SMs
+    const int sms = num_sms_current();
+    int ks = 1;
+    if (pl.grid * 2 <= sms && p.num_kc >= 8) {
+      ks = sms / pl.grid;
+      if (ks > p.num_kc / 4) ks = p.num_kc / 4;
+      if (ks > 16) ks = 16;
+      if (ks < 1) ks = 1;
+    }
+    p.ksplit = ks;
+    pl.grid *= ks;
+  }
   p.z_dbg = z_dbg;
   p.status = dev_status;
   p.timeout_ns = timeout_ns_from_env();
@@ -1070,6 +1095,8 @@ static int launch(const dflash_bf16* H, const dflash_bf16* W, int M, int V, int 
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
+  if (p.ksplit > 1 && cudaMemsetAsync(z_dbg, 0, static_cast<size_t>(M) * V * sizeof(float), st) != cudaSuccess)
+    return DFLASH_ERR_CUDA;
   if (pl.mode == MODE_STREAM)
     e = launch_main<MODE_STREAM, false>(pl, ta, tb, st);
   else

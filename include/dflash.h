@@ -165,7 +165,10 @@ int dflash_lmhead_logits_debug(const dflash_bf16* H, const dflash_bf16* W, int M
  *   C[m,n] = sum_k A[m,k] * B[n,k]      (fp32 accumulation, fp32 out)
  * A [M, K] bf16, B [N, K] bf16 (both K-major, 16-byte aligned), C [M, N] fp32
  * row-major (16-byte aligned).  K % 8 == 0, N >= 16.  Needs no workspace.
- * It computes the projections of the dynamic conv's tap corrections and of
+ * When M <= 128 and N is small next to the SM count, K is split across
+ * CTAs whose fp32 partial sums are added into C (zeroed first on `stream`):
+ * results then agree with the unsplit sum to fp32 rounding, not bit for bit
+ * from run to run.  It computes the projections of the dynamic conv's tap corrections and of
  * the context-gated pair scorer ("DFlash 2: Keep Drafting Parallel",
  * sections "a lightweight local convolution" and "a lightweight path
  * selector").

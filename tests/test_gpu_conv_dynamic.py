@@ -15,7 +15,8 @@ def _bits(a):
     return syn.f32_to_bf16_bits(np.asarray(a, dtype=np.float32))
 
 
-@pytest.mark.parametrize("M,N,K", [(7, 320, 2560), (1, 16, 64), (130, 48, 192), (512, 640, 512), (33, 1000, 128)])
+@pytest.mark.parametrize("M,N,K", [(7, 320, 2560), (1, 16, 64), (130, 48, 192), (512, 640, 512), (33, 1000, 128),
+                                   (1, 16, 8192), (113, 512, 2560), (100, 2000, 1024)])
 def test_gemm_within_bound(M, N, K):
     import block_draft_selection_b200 as bds
     rng = syn.rng_for(M + N + K, "gate")

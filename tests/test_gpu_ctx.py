@@ -162,3 +162,18 @@ def test_ctx_with_verification():
     racc, rnxt = oracle.verify(ref["path_tok"], target)
     np.testing.assert_array_equal(acc[firm], racc[firm])
     np.testing.assert_array_equal(nxt[firm], rnxt[firm])
+
+
+@pytest.mark.parametrize("B,L,V,d,e", [(3, 16, 3000, 256, 64), (5, 1, 2000, 128, 32), (40, 12, 5000, 256, 128)])
+def test_ctx_edge_shapes(B, L, V, d, e):
+    """L = 16 (clusters of 8 CTAs, two tables each), L = 1 (one table, no
+    cluster) and a batch large enough to run one CTA per block."""
+    w = syn.Workload("ctx-edge", B=B, L=L, P=L + 1, d=d, V=V, r=8, sigma=0.3, seed=B + L)
+    Emb, H, Pab, Pg, logp, idx, anchor = _inputs(w, e)
+    for walk in ("maxsum", "greedy"):
+        tok, slot, score, _, tables, _, _ = _run(Emb, H, Pab, Pg, logp, idx, anchor, B, L, V, walk=walk)
+        ref = oracle.ctx_select(logp, idx, Emb, H, Pab, Pg, anchor, B, L, walk=walk)
+        _check_tables(tables, ref["tables"], _table_bound(Emb, H, Pab, Pg, logp, idx, anchor, B, L))
+        firm = ref["margin"] >= 1e-3 if walk == "maxsum" else (ref["margin"] >= 1e-3).all(axis=1)
+        assert firm.mean() > 0.5
+        np.testing.assert_array_equal(slot[firm], ref["path_slot"][firm])

@@ -164,7 +164,7 @@ def _valid_draw(res, u, v, tol):
     return res[v] > 0 and lo <= t + tol * c[-1] and c[v] >= t - tol * c[-1]
 
 
-@pytest.mark.parametrize("B,L,V,T", [(1, 7, 151936, 1.0), (64, 7, 151936, 0.7), (16, 5, 151936, 1.5),
+@pytest.mark.parametrize("B,L,V,T", [(1, 7, 151936, 1.0), (64, 7, 151936, 0.7), (16, 5, 151936, 1.5), (2, 31, 9000, 1.0),
                                      (8, 4, 4096, 1.0), (5, 3, 8193, 1.0), (9, 6, 10001, 1.0),
                                      (3, 16, 20000, 2.0), (32, 1, 30000, 1.0)])
 def test_verify_rejection(B, L, V, T):

@@ -229,7 +229,7 @@ class Step:
         self.cycle, self.conv = cycle, conv
         if conv == "dynamic":
             self.Wc = bds.bf16_tensor(syn.conv_correction(w), dev)
-            self.cws = torch.empty(max(1, int(bds.lib.dflash_conv2tap_dynamic_workspace(w.B, w.P, w.d))),
+            self.cws = torch.empty(max(1, bds.dflash_conv2tap_dynamic_workspace(w.B, w.P, w.d)),
                                    dtype=torch.uint8, device=dev)
         if cycle == "ctx":
             # the pages' context-gated scorer: tied embeddings (the head), e = 256

@@ -14,6 +14,7 @@ from ._binding import (  # noqa: F401
     LIB_PATH,
     dflash_conv2tap,
     dflash_conv2tap_dynamic,
+    dflash_conv2tap_dynamic_workspace,
     dflash_ctx_project,
     dflash_ctx_project_workspace,
     dflash_ctx_walk,

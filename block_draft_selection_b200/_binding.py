@@ -139,6 +139,10 @@ def dflash_gemm_bf16(A, B, C=None, stream=None):
     return C
 
 
+def dflash_conv2tap_dynamic_workspace(B: int, P: int, d: int) -> int:
+    return int(lib.dflash_conv2tap_dynamic_workspace(B, P, d))
+
+
 def dflash_conv2tap_dynamic(x, a0, a1, wc, prev=None, y=None, ws=None, stream=None):
     """Two-tap conv with per-16-channel tap corrections delta = x . Wc^T.
     x [B,P,d], a0/a1 [d], wc [2*d/16, d], prev [B,d] or None: bf16."""
@@ -151,7 +155,7 @@ def dflash_conv2tap_dynamic(x, a0, a1, wc, prev=None, y=None, ws=None, stream=No
         _need(prev, "prev", torch.bfloat16, (B, d))
     y = _out(y, "y", torch.bfloat16, (B, P, d), x.device)
     if ws is None:
-        n = int(lib.dflash_conv2tap_dynamic_workspace(B, P, d))
+        n = dflash_conv2tap_dynamic_workspace(B, P, d)
         if n == 0:
             raise DFlashError("dflash_conv2tap_dynamic_workspace", DFLASH_ERR_INVALID_ARG)
         ws = torch.empty(n, dtype=torch.uint8, device=x.device)

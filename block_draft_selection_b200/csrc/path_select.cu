@@ -15,13 +15,17 @@
 //   1. each CTA gathers the E rows of the positions it scores and the matrix
 //      M into shared memory (bf16, rows padded by 16 bytes so 16-byte loads
 //      of 8 neighbouring rows hit distinct banks);
-//   2. CTA q scores position pairs i = q, q+Q, ...: u_ij = e_{c_ij} M (fp32),
-//      then the 16x16 pair scores, one (j,k) per thread, written straight
+//   2. CTA q scores position pairs i = q, q+Q, ...: u_ij = e_{c_ij} M on the
+//      tensor cores (mma.sync m16n8k16, bf16 in, fp32 out; M staged
+//      transposed; r not a multiple of 16 falls back to CUDA-core FMAs), then
+//      the 16x16 pair scores in fp32, one (j,k) per thread, written straight
 //      into the leader CTA's shared memory (distributed shared memory);
-//   3. after a cluster barrier, warp 0 of the leader walks the scores: lane
-//      (h,k) takes the max over j in half h of delta[j] + S[j,k], one xor-16
-//      shuffle joins the halves, backpointers go to shared memory; then a
-//      16-lane argmax, a backtrack and (optionally) greedy verification.
+//   3. after a cluster barrier, warp 0 of the leader walks the scores
+//      (walk.cuh): lane (h,k) takes the max over j in half h of
+//      delta[j] + S[j,k], one xor-16 shuffle joins the halves, backpointers
+//      go to shared memory; then a 16-lane argmax, a backtrack and
+//      (optionally) greedy verification against target tokens read at the
+//      start.
 //
 // The same kernel also walks from the last verified ("anchor") token, the
 // walk the section describes: greedily following the best successor, or

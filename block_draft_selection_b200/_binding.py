@@ -35,7 +35,7 @@ class DFlashError(RuntimeError):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m block_draft_selection_b200.build` "
+            f"{LIB_PATH} is missing: build it with `python block_draft_selection_b200/build.py` "
             "(this package has no CPU fallback)")
     lib = ctypes.CDLL(LIB_PATH)
     vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t

@@ -1,6 +1,8 @@
 """Build libdflash.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python -m block_draft_selection_b200.build [--force]
+    python block_draft_selection_b200/build.py [--force]
+
+(run as a file: importing the package loads the library this script builds)
 
 The library statically links the CUDA runtime and resolves the driver's
 tensor-map encoder at run time, so it needs no libcuda at link time.

@@ -10,6 +10,18 @@ if ROOT not in sys.path:
 GOLDEN = os.path.join(ROOT, "tests", "golden")
 
 
+def pytest_sessionstart(session):
+    """Build libdflash.so before collection if it is missing (test modules
+    import the package, which loads the library on import)."""
+    import importlib.util
+    path = os.path.join(ROOT, "block_draft_selection_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_dflash_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    if not os.path.exists(mod.LIB):
+        mod.build_library()
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: full-size workloads")

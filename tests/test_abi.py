@@ -18,9 +18,8 @@ def _declared():
 
 @pytest.fixture(scope="module")
 def lib():
-    from block_draft_selection_b200 import build
-    build.build_library()
-    return ctypes.CDLL(build.LIB)
+    from helpers_build import build_library
+    return ctypes.CDLL(build_library())
 
 
 def test_exports_every_declared_symbol(lib):

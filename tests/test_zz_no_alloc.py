@@ -18,9 +18,8 @@ pytestmark = pytest.mark.gpu
 
 
 def _lib():
-    from block_draft_selection_b200 import build
-    build.build_library()
-    lib = ctypes.CDLL(build.LIB)
+    from helpers_build import build_library
+    lib = ctypes.CDLL(build_library())
     vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     lib.dflash_lmhead_topk.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, sz, vp, vp]
     lib.dflash_lmhead_topk_static.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]

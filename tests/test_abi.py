@@ -115,3 +115,11 @@ def test_workspace_rejects_bad_sizes(lib):
     assert lib.dflash_lmhead_topk_workspace(0, 4096, 256) == 0
     assert lib.dflash_lmhead_topk_workspace(4, 8, 256) == 0
     assert lib.dflash_lmhead_topk_workspace(4, 4096, 100) == 0
+
+
+def test_binding_exposes_every_entry_point():
+    """The Python package has a function named after every entry point the
+    header declares (the binding is argument marshalling over the same names)."""
+    import block_draft_selection_b200 as bds
+    missing = [n for n in _declared() if not hasattr(bds, n)]
+    assert not missing, missing

@@ -7,7 +7,9 @@ in Python and checked against a full sort of every candidate (no GPU).
   ranking them under (value desc, index asc) yields the exact top-16;
 - bitonic merge of two sorted 16-lists (the epilogue's half merge): the
   elementwise better of a[k] and b[15-k], then four half-cleaner stages;
-- the 16-element bitonic sorting network that fills an empty list.
+- the 16-element bitonic sorting network that fills an empty list;
+- the weight-streaming tile plan: every tile width a CTA runs is one of the
+  at most four widths the host builds tensor maps for.
 Ties, duplicate values, records with empty slots and few records are all
 exercised; the GPU tests check the kernels themselves."""
 import numpy as np
@@ -128,3 +130,52 @@ def test_bitonic_merge_and_sort_network(seed):
     b = sorted(ents[K:], key=lambda e: _key(*e))
     assert _bitonic_merge(a, b) == sorted(ents, key=lambda e: _key(*e))[:K]
     assert _sort16(ents[:K]) == a
+
+
+def _stream_tiles(units, G, c):
+    """Widths (in rows) of CTA c's tiles: its balanced 16-row-unit range cut
+    into the fewest equal tiles of at most 256 rows."""
+    u0, u1 = c * units // G, (c + 1) * units // G
+    n = u1 - u0
+    nt = -(-n // 16)
+    wu = -(-n // nt) if nt else 0
+    out = []
+    for k in range(nt):
+        t0 = (u0 + k * wu) * 16
+        if t0 >= u1 * 16:
+            break
+        out.append(min(wu * 16, u1 * 16 - t0))
+    return out
+
+
+def _stream_widths(units, G):
+    """The widths the host enumerates (one tensor map each, at most four)."""
+    ws = []
+    u_lo = units // G
+    for u in (u_lo, u_lo + 1):
+        if u < 1:
+            continue
+        nt = -(-u // 16)
+        wu = -(-u // nt)
+        for w in (16 * wu, 16 * (u - (nt - 1) * wu)):
+            if w > 0 and w not in ws:
+                ws.append(w)
+    return ws
+
+
+@pytest.mark.parametrize("V", [16, 17, 100, 4096, 8193, 20000, 129280, 151936, 151937, 256000, 500000])
+def test_stream_tile_widths_are_enumerated(V):
+    """Every tile a CTA runs has one of the (at most four) enumerated widths,
+    the tiles of all CTAs cover the 16-row units exactly once, and none is
+    wider than 256 rows."""
+    units = -(-V // 16)
+    for sms in (148, 132, 8):
+        G = min(units, sms)
+        ws = _stream_widths(units, G)
+        assert len(ws) <= 4
+        covered = 0
+        for c in range(G):
+            tiles = _stream_tiles(units, G, c)
+            assert all(w in ws and 0 < w <= 256 for w in tiles)
+            covered += sum(tiles)
+        assert covered == units * 16

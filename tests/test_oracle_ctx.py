@@ -1,7 +1,9 @@
 """Pins for the oracle's context-gated scorer (no GPU): a hand-worked case,
-exact rational tables with the gate fixed at 1/2 (zero gate projection) and
-at 1 (saturated gate), brute force over every anchored path, the zero
-projection case and a planted swap of the two projections."""
+exact rational tables with the gate fixed at 1/2 (zero gate projection), at 1
+(saturated gate) and switching between 1 and 0 from one position to the next
+(which hidden state gates which table), brute force over every anchored path,
+the zero projection case and planted slips (the two projections swapped; the
+gate taken from the neighbouring position)."""
 import itertools
 from fractions import Fraction
 
@@ -61,7 +63,9 @@ def _random(seed, B, L, V, d, e, gate_scale):
 
 
 def _exact_tables(logp, idx, Emb, Pab, anchor, b, L, e, gate):
-    """Tables from Fractions of the bit patterns, with a fixed gate value."""
+    """Tables from Fractions of the bit patterns, with a fixed gate value
+    (one Fraction for every table, or a list: table t gated by gate[t])."""
+    gates = list(gate) if isinstance(gate, (list, tuple)) else [gate] * L
     d = Emb.shape[1]
     proj = lambda tok, rows: [sum(bf(Emb[tok, c]) * bf(Pab[q, c]) for c in range(d)) for q in rows]
     A = lambda tok: proj(tok, range(e))
@@ -71,7 +75,7 @@ def _exact_tables(logp, idx, Emb, Pab, anchor, b, L, e, gate):
     for t in range(L):
         preds = [A(int(anchor[b]))] * K if t == 0 else [A(int(idx[b * L + t - 1, j])) for j in range(K)]
         succ = [Bp(int(idx[b * L + t, k])) for k in range(K)]
-        T.append([[lp(t, k) + sum(preds[j][q] * gate * succ[k][q] for q in range(e)) for k in range(K)]
+        T.append([[lp(t, k) + sum(preds[j][q] * gates[t] * succ[k][q] for q in range(e)) for k in range(K)]
                   for j in range(K)])
     return T
 
@@ -139,3 +143,52 @@ def test_gate_is_a_sigmoid():
     np.testing.assert_allclose(oracle.ctx_scorer.sigmoid(x) + oracle.ctx_scorer.sigmoid(-x), 1.0, rtol=0,
                                atol=1e-15)
     assert oracle.ctx_scorer.sigmoid(np.log(3.0)) == pytest.approx(0.75, rel=1e-15)
+
+
+def _alternating_gate_case(L, seed):
+    """Hidden states +1 at even positions and -1 at odd ones with Pg = 64
+    everywhere (d = 8): Pg.h_t = +-512, so the gate is 1 at even t and
+    sigmoid(-512) ~ 4e-223 (0 to far below any tolerance) at odd t."""
+    B, V, d, e = 2, 150, 8, 4
+    logp, idx, Emb, _, Pab, _, anchor = _random(seed, B, L, V, d, e, 0.0)
+    sign = np.where(np.arange(B * L) % L % 2 == 0, 1.0, -1.0).astype(np.float32)
+    H = f32_to_bf16_bits(sign[:, None] * np.ones((B * L, d), np.float32))
+    Pg = f32_to_bf16_bits(np.full((e, d), 64.0, np.float32))
+    gates = [Fraction(1) if t % 2 == 0 else Fraction(0) for t in range(L)]
+    return B, e, logp, idx, Emb, H, Pab, Pg, anchor, gates
+
+
+def _as_float(T):
+    return np.array([[[float(x) for x in r] for r in Tt] for Tt in T])
+
+
+@pytest.mark.parametrize("L,seed", [(3, 11), (4, 12)])
+def test_gate_follows_own_position(L, seed):
+    """Table t is gated by the hidden state at position t: with gates that
+    alternate 1, 0, 1, ... the tables equal the exact rational ones whose
+    table t carries the gate of position t (S_t(a, b) = U_t(b) +
+    <A(a) (.) H(h_t), B(b)>, "DFlash 2: Keep Drafting Parallel", section "a
+    lightweight path selector")."""
+    B, e, logp, idx, Emb, H, Pab, Pg, anchor, gates = _alternating_gate_case(L, seed)
+    T = oracle.ctx_tables(logp, idx, Emb, H, Pab, Pg, anchor, B, L)
+    for b in range(B):
+        ex = _as_float(_exact_tables(logp, idx, Emb, Pab, anchor, b, L, e, gates))
+        np.testing.assert_allclose(T[b], ex, rtol=1e-13, atol=1e-12)
+        # the gated-off tables are the unary term alone
+        for t in range(1, L, 2):
+            np.testing.assert_allclose(T[b, t], np.broadcast_to(logp[b * L + t].astype(np.float64), (K, K)),
+                                       rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("shift", [1, -1])
+def test_planted_gate_position_slip_is_caught(shift):
+    """Gating table t with h_{t-1} (shift 1) or h_{t+1} (shift -1): the same
+    oracle fed hidden states moved by one position (a copy, on the CPU) gives
+    tables that miss the exact ones by far more than any tolerance."""
+    L = 4
+    B, e, logp, idx, Emb, H, Pab, Pg, anchor, gates = _alternating_gate_case(L, 13)
+    Hs = np.roll(H.reshape(B, L, -1), shift, axis=1).reshape(B * L, -1)
+    wrong = oracle.ctx_tables(logp, idx, Emb, Hs, Pab, Pg, anchor, B, L)
+    for b in range(B):
+        ex = _as_float(_exact_tables(logp, idx, Emb, Pab, anchor, b, L, e, gates))
+        assert np.abs(wrong[b] - ex).max() > 1e-3

@@ -30,6 +30,7 @@ from ._binding import (  # noqa: F401
     dflash_lmhead_topk_partial,
     dflash_lmhead_topk_records,
     dflash_status_string,
+    dflash_build_id,
     dflash_verify,
     dflash_verify_rejection,
     dflash_verify_rejection_workspace,

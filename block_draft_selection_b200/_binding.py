@@ -41,6 +41,7 @@ def _load():
     vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     sig = {
         "dflash_status_string": (ctypes.c_char_p, [i32]),
+        "dflash_build_id": (ctypes.c_char_p, []),
         "dflash_conv2tap": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, vp]),
         "dflash_lmhead_topk_workspace": (sz, [i32, i32, i32]),
         "dflash_lmhead_topk": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, sz, vp, vp]),
@@ -69,7 +70,25 @@ def _load():
         f = getattr(lib, name)
         f.restype = res
         f.argtypes = args
+    _check_build_id(lib)
     return lib
+
+
+def _check_build_id(lib):
+    """Refuse a library compiled from other sources than the ones beside it
+    (when the sources are present): stale native code must not pass for the
+    current code."""
+    build_py = os.path.join(os.path.dirname(LIB_PATH), "build.py")
+    if not os.path.isdir(os.path.join(os.path.dirname(LIB_PATH), "csrc")) or not os.path.exists(build_py):
+        return
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("_dflash_build_check", build_py)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    have, want = lib.dflash_build_id().decode(), mod.source_hash()
+    if have != want:
+        raise ImportError(f"{LIB_PATH} was built from other sources (build id {have}, sources {want}): "
+                          "rebuild it with `python block_draft_selection_b200/build.py`")
 
 
 lib = _load()
@@ -77,6 +96,10 @@ lib = _load()
 
 def dflash_status_string(code: int) -> str:
     return lib.dflash_status_string(int(code)).decode()
+
+
+def dflash_build_id() -> str:
+    return lib.dflash_build_id().decode()
 
 
 def _check(fn: str, code: int):

@@ -6,8 +6,16 @@
 
 The library statically links the CUDA runtime and resolves the driver's
 tensor-map encoder at run time, so it needs no libcuda at link time.
+
+Staleness is decided by content, not by file times: a SHA-256 over the
+sources' paths and bytes is compiled into the library (dflash_build_id())
+and written beside it (libdflash.so.srchash); a library whose recorded hash
+differs from the current sources is rebuilt.  A copied tree, a checkout that
+resets mtimes, or a prebuilt library carried along with other sources can
+therefore never stand in for the sources at hand.
 """
 import glob
+import hashlib
 import os
 import shutil
 import subprocess
@@ -18,6 +26,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libdflash.so")
+HASH_FILE = LIB + ".srchash"
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr"]
@@ -38,24 +47,45 @@ def _inputs():
     return sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
 
 
+def source_hash() -> str:
+    """First 16 hex digits of a SHA-256 over every input's path (relative to
+    the repository) and bytes, in sorted path order, plus the compile flags."""
+    h = hashlib.sha256()
+    for f in sorted(_inputs()):
+        h.update(os.path.relpath(f, ROOT).replace(os.sep, "/").encode() + b"\0")
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+        h.update(b"\0")
+    h.update(" ".join(ARCH + FLAGS).encode())
+    return h.hexdigest()[:16]
+
+
+def recorded_hash():
+    try:
+        with open(HASH_FILE) as f:
+            return f.read().strip()
+    except OSError:
+        return None
+
+
 def up_to_date() -> bool:
-    if not os.path.exists(LIB):
-        return False
-    t = os.path.getmtime(LIB)
-    return all(os.path.getmtime(f) <= t for f in _inputs())
+    return os.path.exists(LIB) and recorded_hash() == source_hash()
 
 
 def build_library(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
+    digest = source_hash()
     tmp = LIB + ".tmp"
-    cmd = [_nvcc(), *ARCH, *FLAGS, "-I", INCLUDE, "-o", tmp, *sources()]
+    cmd = [_nvcc(), *ARCH, *FLAGS, f"-DDFLASH_SOURCE_HASH=\"{digest}\"", "-I", INCLUDE, "-o", tmp, *sources()]
     if verbose:
         print(" ".join(cmd), flush=True)
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + r.stdout + r.stderr)
     os.replace(tmp, LIB)
+    with open(HASH_FILE, "w") as f:
+        f.write(digest + "\n")
     return LIB
 
 

@@ -1,5 +1,11 @@
-// Status strings of the C ABI.
+// Status strings and the build identity of the C ABI.
 #include "../../include/dflash.h"
+
+#ifndef DFLASH_SOURCE_HASH
+#define DFLASH_SOURCE_HASH "unhashed"
+#endif
+
+extern "C" const char* dflash_build_id(void) { return DFLASH_SOURCE_HASH; }
 
 extern "C" const char* dflash_status_string(int status) {
   switch (status) {

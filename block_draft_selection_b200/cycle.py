@@ -7,10 +7,11 @@ inputs from pinned host buffers to the device, runs the cycle and copies its
 results back, all captured once into a CUDA graph so a step costs one graph
 launch on the host.  Weights (W, E, M, conv taps) stay on the device.
 
-The step's inputs live in one pinned host arena and one device arena with the
-same layout (each tensor at a 256-byte-aligned offset), and so do its results:
-a step moves its inputs with one host-to-device copy and its results with one
-device-to-host copy.
+The step's inputs, a status word and its results live in one device buffer
+(each tensor at a 256-byte-aligned offset), mirrored by a pinned host buffer
+for the inputs and one for the results: a step moves its inputs (and a zero
+status word) with one host-to-device copy and the status word and its results
+with one device-to-host copy, and `run()` raises if the status is nonzero.
 """
 from __future__ import annotations
 
@@ -19,26 +20,51 @@ import torch
 from . import _binding as b
 
 
-def _arena(specs, device, pinned=False, align=256):
-    """One byte buffer holding tensors of the given (name, shape, dtype) at
-    aligned offsets; returns (buffer, {name: view})."""
+def _nbytes(shape, dt) -> int:
+    n = 1
+    for x in shape:
+        n *= x
+    return n * torch.tensor([], dtype=dt).element_size()
+
+
+def _offsets(specs, align=256):
+    """Offsets of (name, shape, dtype) tensors packed in order at `align`-byte
+    boundaries: ({name: (offset, shape, dtype)}, end)."""
     offs, off = {}, 0
     for name, shape, dt in specs:
         off = (off + align - 1) // align * align
-        n = 1
-        for x in shape:
-            n *= x
         offs[name] = (off, shape, dt)
-        off += n * torch.tensor([], dtype=dt).element_size()
-    buf = torch.empty(max(off, 1), dtype=torch.uint8, device=device, pin_memory=pinned)
-    views = {}
-    for name, (o, shape, dt) in offs.items():
-        n = 1
-        for x in shape:
-            n *= x
-        nb = n * torch.tensor([], dtype=dt).element_size()
-        views[name] = buf[o:o + nb].view(dt).view(shape)
-    return buf, views
+        off += _nbytes(shape, dt)
+    return offs, off
+
+
+def _views(buf, offs, names, base=0):
+    """Typed views of `buf` (a uint8 buffer that starts at byte `base` of the
+    layout) for the listed names."""
+    out = {}
+    for name in names:
+        o, shape, dt = offs[name]
+        out[name] = buf[o - base:o - base + _nbytes(shape, dt)].view(dt).view(shape)
+    return out
+
+
+def _arena(specs, device, pinned=False, align=256):
+    """One byte buffer holding tensors of the given (name, shape, dtype) at
+    aligned offsets; returns (buffer, {name: view})."""
+    offs, end = _offsets(specs, align)
+    buf = torch.empty(max(end, 1), dtype=torch.uint8, device=device, pin_memory=pinned)
+    return buf, _views(buf, offs, [n for n, _, _ in specs])
+
+
+def io_layout(ins, outs):
+    """Layout of a step's device buffer: the inputs, the status word, then the
+    results.  The host-to-device copy covers [0, in_end) -- inputs and the
+    status word, which the host side keeps at zero, so each step starts with
+    a cleared status -- and the device-to-host copy covers [out_begin, end) --
+    the status word and the results.  Returns (offsets, in_end, out_begin, end)."""
+    offs, end = _offsets(list(ins) + [("status", (1,), torch.int32)] + list(outs))
+    s_off = offs["status"][0]
+    return offs, s_off + 4, s_off, end
 
 
 class DraftCycle:
@@ -53,16 +79,23 @@ class DraftCycle:
                ("target", (B, L + 1), torch.int32)]
         outs = [("path_tok", (B, L), torch.int32), ("accept_len", (B,), torch.int32),
                 ("next_token", (B,), torch.int32), ("y", (B, P, d), torch.bfloat16)]
-        # device arenas (inputs, results) and their pinned host twins
-        self._din, din = _arena(ins, dev)
-        self._dout, dout = _arena(outs, dev)
-        self._hin, self.host_in = _arena(ins, "cpu", pinned=True)
-        self._hout, self.host_out = _arena(outs, "cpu", pinned=True)
-        self.H, self.x, self.prev, self.target = din["H"], din["x"], din["prev"], din["target"]
-        self.tok, self.acc, self.nxt, self.y = dout["path_tok"], dout["accept_len"], dout["next_token"], dout["y"]
+        # one device buffer (inputs | status | results) and pinned host twins
+        # of its input span and its result span
+        offs, in_end, out_begin, end = io_layout(ins, outs)
+        in_names = [n for n, _, _ in ins] + ["status"]
+        out_names = ["status"] + [n for n, _, _ in outs]
+        self._dbuf = torch.zeros(end, dtype=torch.uint8, device=dev)
+        dv = _views(self._dbuf, offs, in_names + out_names[1:])
+        self._din, self._dout = self._dbuf[:in_end], self._dbuf[out_begin:]
+        self._hin = torch.zeros(in_end, dtype=torch.uint8, pin_memory=True)    # its status word stays 0
+        self._hout = torch.zeros(end - out_begin, dtype=torch.uint8, pin_memory=True)
+        self.host_in = _views(self._hin, offs, in_names[:-1])
+        self.host_out = _views(self._hout, offs, out_names, base=out_begin)
+        self.H, self.x, self.prev, self.target = dv["H"], dv["x"], dv["prev"], dv["target"]
+        self.tok, self.acc, self.nxt, self.y = dv["path_tok"], dv["accept_len"], dv["next_token"], dv["y"]
         self.lp, self.ix, self.lse = e((M, 16), torch.float32), e((M, 16), torch.int32), e((M,), torch.float32)
         self.slot, self.score = e((B, L), torch.int32), e((B,), torch.float32)
-        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.status = dv["status"]
         self.ws = b.workspace(M, V, d, dev)
         self._graph = None
         if use_graph:
@@ -94,12 +127,18 @@ class DraftCycle:
         torch.cuda.current_stream().wait_stream(side)
 
     def run(self):
-        """One step: host inputs (self.host_in) -> device -> cycle -> host results."""
+        """One step: host inputs (self.host_in) -> device -> cycle -> host
+        results.  Raises DFlashError when a kernel of the step recorded a
+        device-side error (a bounded wait that ran out, a token index out of
+        range): the results of such a step are not valid."""
         if self._graph is not None:
             self._graph.replay()
         else:
             self._step()
         torch.cuda.current_stream().synchronize()
+        code = int(self.host_out["status"][0])
+        if code != 0:
+            raise b.DFlashError("DraftCycle.run", code)
         return self.host_out
 
     def io_bytes(self):

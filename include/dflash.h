@@ -58,6 +58,13 @@ enum dflash_status {
 /* Static text for a status code (never NULL). */
 const char* dflash_status_string(int status);
 
+/* Identity of the sources this library was compiled from: the first 16 hex
+ * digits of a SHA-256 over the CUDA sources, headers and compile flags
+ * (computed by the package's build script), or "unhashed" for a build made
+ * without it.  Static text, never NULL; no GPU is touched.  The library's
+ * own bookkeeping, not a computation of the pages, so it cites none. */
+const char* dflash_build_id(void);
+
 /*
  * Two-tap block-local convolution.
  * "DFlash 2: Keep Drafting Parallel", section "a lightweight local

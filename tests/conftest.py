@@ -11,15 +11,17 @@ GOLDEN = os.path.join(ROOT, "tests", "golden")
 
 
 def pytest_sessionstart(session):
-    """Build libdflash.so before collection if it is missing (test modules
-    import the package, which loads the library on import)."""
+    """Build libdflash.so before collection unless the library present was
+    compiled from exactly these sources (test modules import the package,
+    which loads the library on import).  The check compares a hash of the
+    sources with the one recorded at build time, so a library left over from
+    other sources is rebuilt rather than tested."""
     import importlib.util
     path = os.path.join(ROOT, "block_draft_selection_b200", "build.py")
     spec = importlib.util.spec_from_file_location("_dflash_build", path)
     mod = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(mod)
-    if not os.path.exists(mod.LIB):
-        mod.build_library()
+    mod.build_library()
 
 
 def pytest_configure(config):

@@ -29,6 +29,25 @@ def test_exports_every_declared_symbol(lib):
         assert hasattr(lib, n), n
 
 
+def test_build_id_matches_sources(lib):
+    """The library loaded here was compiled from the sources in this tree."""
+    from helpers_build import build_module
+    lib.dflash_build_id.restype = ctypes.c_char_p
+    assert lib.dflash_build_id().decode() == build_module().source_hash()
+
+
+def test_stale_library_is_rebuilt(tmp_path, monkeypatch):
+    """A recorded hash that differs from the sources' hash means the library
+    is out of date, whatever the files' modification times say."""
+    mod = __import__("helpers_build").build_module()
+    stamp = tmp_path / "stamp"
+    stamp.write_text("0123456789abcdef\n")
+    monkeypatch.setattr(mod, "HASH_FILE", str(stamp))
+    assert not mod.up_to_date()
+    stamp.write_text(mod.source_hash() + "\n")
+    assert mod.up_to_date() == os.path.exists(mod.LIB)
+
+
 def test_status_strings(lib):
     lib.dflash_status_string.restype = ctypes.c_char_p
     seen = set()

@@ -11,10 +11,18 @@ tokens.  Inputs are seeded synthetic arrays of the workload's shapes and
 distributions (block_draft_synth); W alone is larger than L2, so steps do not
 reuse each other's data through L2.
 
-Multi-GPU: one process per GPU (torchrun); blocks are independent, so each
-rank runs its own batch with replicated weights and no data-path collective
-(weak scaling).  The timed region is bracketed by a barrier and a device
-synchronize; the elapsed device time is the max over ranks.
+The printed line is the headline workload (default: throughput, 256 blocks of
+16 positions, d = 4096, V = 129,280 -- the largest of the five); with one GPU
+the same run also times every other workload for its own K steps and reports
+each under "workloads", with its own roofline, stage times, clocks and
+end-to-end figure.
+
+Multi-GPU: one process per GPU.  `--gpus N` outside torchrun starts N ranks
+itself through torch.distributed.run on 127.0.0.1; under torchrun WORLD_SIZE
+must equal N.  Blocks are independent, so each rank runs its own batch with
+replicated weights and no data-path collective (weak scaling).  The timed
+region is bracketed by a barrier and a device synchronize; the elapsed device
+time is the max over ranks.
 
 `--impl reference` times the CPU oracle (float64 numpy) on the host's cores on
 a bounded sample of the same workload; it is a deliberately slow baseline.
@@ -26,6 +34,7 @@ import hashlib
 import json
 import os
 import statistics
+import subprocess
 import sys
 import threading
 import time
@@ -40,7 +49,7 @@ import block_draft_synth as syn  # noqa: E402
 
 METRIC = "draft blocks/sec (LM-head+top16+select+verify) on 1 B200; % of roofline"
 UNIT = "blocks/s"
-DEFAULT_WORKLOAD = "qwen3-4b-bs1"
+DEFAULT_WORKLOAD = "throughput"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
@@ -253,12 +262,6 @@ class Step:
 
     # conv, LM-head GEMM+epilogue, LM-head merge, select+verify
     LAUNCHES_PER_STEP = 4
-    STAGES = ("conv2tap", "lmhead_topk", "select_verify")
-    # "lmhead_select" brackets the LM head and the selection stage of one
-    # cycle together: minus the LM head's own bracket it is the time the
-    # selection stage adds to a cycle, with the selector's launch allowed to
-    # overlap the end of the LM head as it does in untimed cycles
-    TIMED = STAGES + ("event_pair", "lmhead_select")
     # sample cycle: conv, LM head (2), walk, rejection verification (2)
     LAUNCHES_PER_STEP_SAMPLE = 6
     # ctx cycle: conv, LM head (2), projections (gather + 2 GEMMs), scores + walk
@@ -271,7 +274,9 @@ class Step:
 
     def run(self, marks=None):
         """One cycle.  `marks`: optional {stage name: (event, event)} recorded
-        around that stage's call."""
+        around that stage's call; "event_pair" brackets nothing (the cost of
+        the two event nodes) and "lmhead_select" brackets the LM head and the
+        selection stage together."""
         bds = self.bds
         marks = marks or {}
 
@@ -322,18 +327,14 @@ class Step:
             span[1].record()
 
 
-def _graph_steps(step, n_steps):
-    """Capture n_steps cycles into one CUDA graph.  Up to three of them carry
-    external timing events (event nodes) around one stage each -- the last
-    cycle around the LM head, the one before around select+verify, the one
-    before that around the conv -- so stage durations are sampled inside the
-    timed region at a cost of a few event nodes per graph."""
+def _graph_steps(step, n_steps, plan):
+    """Capture n_steps cycles into one CUDA graph.  plan(k) names the stage
+    whose call cycle k brackets with a pair of external timing events (event
+    nodes), or None.  Returns (graph, [(stage name, (start, end))])."""
     import torch
     ev = lambda: (torch.cuda.Event(enable_timing=True, external=True),
                   torch.cuda.Event(enable_timing=True, external=True))
-    plan = {n_steps - 1: "lmhead_topk", n_steps - 2: "select_verify", n_steps - 3: "conv2tap",
-            n_steps - 4: "event_pair", n_steps - 5: "lmhead_select"}
-    marks = {k: {name: ev()} for k, name in plan.items() if k >= 0}
+    marks = [{plan(k): ev()} if plan(k) else None for k in range(n_steps)]
     g = torch.cuda.CUDAGraph()
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
@@ -342,10 +343,10 @@ def _graph_steps(step, n_steps):
     side.synchronize()
     with torch.cuda.graph(g, stream=side):
         for k in range(n_steps):
-            step.run(marks.get(k))
+            step.run(marks[k])
     torch.cuda.current_stream().wait_stream(side)
     torch.cuda.synchronize()
-    return g, {name: pair for m in marks.values() for name, pair in m.items()}
+    return g, [(name, pair) for m in marks if m for name, pair in m.items()]
 
 
 def _chunk(steps, cap=32):
@@ -353,19 +354,52 @@ def _chunk(steps, cap=32):
     return max(c for c in range(1, min(cap, steps) + 1) if steps % c == 0)
 
 
-def gpu_arm(args, w: syn.Workload):
+# Stage breakdown: one extra graph after the timed region in which cycle k
+# brackets stage BREAKDOWN[k % 5]; every stage gets BREAKDOWN_SAMPLES samples.
+BREAKDOWN = ("event_pair", "conv2tap", "lmhead_topk", "select_verify", "lmhead_select")
+BREAKDOWN_SAMPLES = 24
+
+
+def _summ(xs):
+    xs = sorted(xs)
+    return {"mean": statistics.mean(xs), "median": statistics.median(xs), "min": xs[0], "max": xs[-1],
+            "n": len(xs)} if xs else None
+
+
+def _release():
+    import gc
+    import torch
+    gc.collect()
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def _calibrated_steps(step, target_s: float, floor: int, cap: int = 20000) -> int:
+    """Cycles that make a timed region of about target_s seconds (at least
+    `floor`), from one replay of an 8-cycle graph; a multiple of 32 when
+    that many."""
+    import torch
+    g, _ = _graph_steps(step, 8, lambda k: None)
+    g.replay()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(3):
+        g.replay()
+    t1.record()
+    torch.cuda.synchronize()
+    per = t0.elapsed_time(t1) / 1e3 / 24
+    del g
+    n = int(min(cap, max(floor, target_s / max(per, 1e-9))))
+    return n - n % 32 if n >= 64 else n
+
+
+def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, device):
+    """Time `steps` cycles of workload w (steps None: calibrated to about
+    args.sub_seconds, at least args.steps) and return the workload's result:
+    blocks/s, the LM head's roofline from the timed region, the stage
+    breakdown, clocks and the end-to-end figure."""
     import torch
     import block_draft_selection_b200 as bds
-    rank, local_rank, world = dist_env()
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
-                                device_id=torch.device("cuda", local_rank))
-    device = torch.device("cuda", local_rank)
-    torch.cuda.set_device(device)
-    step = Step(w, rank, device, args.cycle, args.conv)
 
     def barrier():
         torch.cuda.synchronize()
@@ -374,25 +408,30 @@ def gpu_arm(args, w: syn.Workload):
             dist.barrier()
         torch.cuda.synchronize()
 
-    for _ in range(args.warmup):
+    step = Step(w, rank, device, args.cycle, args.conv)
+    for _ in range(warmup):
         step.run()
+    torch.cuda.synchronize()
+    if steps is None:
+        steps = _calibrated_steps(step, args.sub_seconds, args.steps)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    samples = {n: [] for n in Step.TIMED}
+    # timed region: every cycle brackets its LM-head call, so the roofline's
+    # launch duration is sampled live in the timed region (one sample per step)
     if args.eager:
         chunk, graphs = 1, []
-        marks = [{n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for n in Step.TIMED} for _ in range(args.steps)]
+        marks = [{"lmhead_topk": (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))}
+                 for _ in range(steps)]
     else:
-        chunk = _chunk(args.steps)
-        n_rep = args.steps // chunk
-        graphs = [_graph_steps(step, chunk) for _ in range(min(8, n_rep))]
+        chunk = _chunk(steps)
+        n_rep = steps // chunk
+        graphs = [_graph_steps(step, chunk, lambda k: "lmhead_topk") for _ in range(min(8, n_rep))]
         for g, _ in graphs:
             g.replay()              # one untimed replay of each captured graph
     barrier()
     with ClockSampler(device.index if device.index is not None else 0) as clk:
         t0.record()
         if args.eager:
-            for k in range(args.steps):
+            for k in range(steps):
                 step.run(marks[k])
         else:
             for rep in range(n_rep):
@@ -401,62 +440,70 @@ def gpu_arm(args, w: syn.Workload):
         torch.cuda.synchronize()
     barrier()
     if int(step.status.item()) != 0:
-        raise RuntimeError(f"device status {int(step.status.item())} during the timed region")
+        raise RuntimeError(f"device status {int(step.status.item())} during the timed region ({w.name})")
     ms = t0.elapsed_time(t1)
-    # stage durations: every cycle of the eager loop, or the instrumented cycles
-    # of each graph's last replay inside the timed region
-    for m in (marks if args.eager else [gm for _, gm in graphs]):
-        for n, (a, b) in m.items():
-            samples[n].append(a.elapsed_time(b))
-    mean = lambda n: statistics.mean(samples[n]) if samples[n] else float("nan")
-    ev_ms = mean("event_pair") if samples["event_pair"] else 0.0
-    raw_ms = [mean(n) for n in Step.STAGES]
-    # net of the two event nodes that bracket each timed stage
-    stage_ms = [max(0.0, t - ev_ms) for t in raw_ms]
-    lm_ms = raw_ms[1]                   # gross: includes the bracketing event nodes (conservative)
-    lm_net_ms = stage_ms[1]
-    # time the selection stage adds to a cycle (both brackets gross, so the
-    # event-node cost cancels)
-    span_ms = mean("lmhead_select") if samples["lmhead_select"] else float("nan")
-    sel_added_ms = max(0.0, span_ms - lm_ms) if span_ms == span_ms else None
+    # LM-head launch durations of the timed region: every cycle of the eager
+    # loop, or every cycle of each graph's last replay
+    if args.eager:
+        lm_samples = [m["lmhead_topk"][0].elapsed_time(m["lmhead_topk"][1]) for m in marks]
+    else:
+        lm_samples = [a.elapsed_time(b) for _, gm in graphs for _, (a, b) in gm]
     ms_max = reduce_max(ms, world)
-    value = aggregate(w.B, world, ms_max, args.steps)
+    value = aggregate(w.B, world, ms_max, steps)
     del graphs
+
+    # stage breakdown (after the timed region, same clocks regime): cycle k of
+    # one graph brackets stage BREAKDOWN[k % 5]
+    sg, sm = _graph_steps(step, len(BREAKDOWN) * BREAKDOWN_SAMPLES, lambda k: BREAKDOWN[k % len(BREAKDOWN)])
+    sg.replay()
+    torch.cuda.synchronize()
+    if int(step.status.item()) != 0:
+        raise RuntimeError(f"device status {int(step.status.item())} in the stage breakdown ({w.name})")
+    samples = {n: [] for n in BREAKDOWN}
+    for name, (a, b) in sm:
+        samples[name].append(a.elapsed_time(b))
+    del sg, sm
+    med = lambda n: statistics.median(samples[n])
+    ev_ms = med("event_pair")
+    stage_ms = {n: max(0.0, med(n) - ev_ms) for n in ("conv2tap", "lmhead_topk", "select_verify")}
+    # what the selection stage adds to a cycle: (LM head + selection bracketed
+    # together) - (LM head bracketed alone); both gross, the event cost cancels
+    sel_added_ms = max(0.0, med("lmhead_select") - med("lmhead_topk"))
+    cyc_ms = ms_max / steps
 
     # end-to-end leg: the library's DraftCycle, one graph launch per step that
     # copies the step's inputs from pinned host memory, runs the cycle and
     # copies the results back; the host waits for them every step
-    e2e = None
     if args.cycle == "greedy" and args.conv == "static":
         cyc = bds.DraftCycle(step.W, step.E, step.Msel, step.a0, step.a1, w.B, w.L, w.P)
         cyc.host_in["H"].copy_(step.H)
         cyc.host_in["x"].copy_(step.x)
         cyc.host_in["prev"].copy_(step.prev)
         cyc.host_in["target"].copy_(step.target)
-        for _ in range(max(3, args.warmup // 2)):
+        for _ in range(max(3, warmup)):
             cyc.run()
         barrier()
-        e_steps = max(1, args.steps)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        for _ in range(e_steps):
-            cyc.run()
+        for _ in range(steps):
+            cyc.run()               # raises if a kernel of the step reports a device error
         e1.record()
         torch.cuda.synchronize()
         barrier()
-        if int(cyc.status.item()) != 0:
-            raise RuntimeError(f"device status {int(cyc.status.item())} in the end-to-end leg")
         e_ms = reduce_max(e0.elapsed_time(e1), world)
         h2d, d2h = cyc.io_bytes()
-        e2e = {"value": aggregate(w.B, world, e_ms, e_steps), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "path": "DraftCycle.run(): pinned H2D + conv + LM head + select/verify + D2H, host sync"}
+        e2e = {"value": aggregate(w.B, world, e_ms, steps), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+               "path": "DraftCycle.run(): pinned H2D + conv + LM head + select/verify + D2H (with the status word), "
+                       "host sync"}
+        del cyc
     else:
         e2e = {"value": None, "unit": UNIT, "h2d_bytes_per_step": None, "d2h_bytes_per_step": None,
                "path": "measured for the greedy cycle with static taps only (the metric's path)"}
 
     peaks, peaks_kind = load_peaks()
     alg_bytes, alg_flops = lmhead_algorithmic(w)
+    lm_ms = statistics.mean(lm_samples)
     t_lm = lm_ms / 1e3
     hbm_t = alg_bytes / (peaks["hbm_gbs"] * 1e9)
     tc_t = alg_flops / (peaks["bf16_tflops"] * 1e12)
@@ -476,41 +523,72 @@ def gpu_arm(args, w: syn.Workload):
     roof["kernel"] = "dflash_lmhead_topk (GEMM+epilogue and merge kernels)"
     roof["algorithmic_per_launch"] = alg_bytes if roof["bound"] == "hbm" else alg_flops
     roof["launch_ms"] = lm_ms
-    roof["launch_ms_net_of_events"] = lm_net_ms
-    roof["frac_net_of_events"] = roof["frac"] * lm_ms / lm_net_ms if lm_net_ms > 0 else None
+    roof["launch_ms_samples"] = _summ(lm_samples)
+    roof["launch_ms_net_of_events"] = max(1e-9, lm_ms - ev_ms)
+    roof["frac_net_of_events"] = roof["frac"] * lm_ms / roof["launch_ms_net_of_events"]
+    roof["timing"] = ("mean CUDA-event duration of the LM-head call (GEMM+epilogue kernel and merge kernel, "
+                      "bracketed by event nodes in every cycle of the timed graphs), over the timed region")
+    stages = {**{n: 1e3 * stage_ms[n] for n in stage_ms},
+              "select_verify_share": stage_ms["select_verify"] / cyc_ms,
+              "select_verify_added": 1e3 * sel_added_ms,
+              "select_verify_added_share": sel_added_ms / cyc_ms,
+              "event_pair_overhead": 1e3 * ev_ms,
+              "samples": {n: len(samples[n]) for n in BREAKDOWN},
+              "raw_us": {n: {k: (1e3 * v if k != "n" else v) for k, v in _summ(samples[n]).items()}
+                         for n in BREAKDOWN},
+              "note": ("medians over one extra graph after the timed region whose cycle k brackets stage "
+                       "k mod 5 (%d samples per stage), net of the bracketing event-node pair (measured alone); "
+                       "select_verify_added = (LM head + selection bracketed together) - (LM head bracketed "
+                       "alone): what the selection stage adds to a cycle when its launch may overlap the LM "
+                       "head's end" % BREAKDOWN_SAMPLES)}
+    config = {"workload": w.name + {"greedy": "", "sample": "+sampled-walk(T=1)",
+                                    "ctx": "+context-gated-scorer"}[args.cycle]
+                          + ("+dynamic-conv" if args.conv == "dynamic" else ""),
+              "blocks_per_gpu": w.B, "L": w.L, "M": w.M, "d": w.d, "V": w.V,
+              "K": 16, "r": w.r, "conv": [w.B, w.P, w.d], "conv_taps": args.conv, "cycle": args.cycle,
+              "parallelism": f"dp{world} (blocks)",
+              "launch": "eager" if args.eager else f"cuda graphs of {chunk} cycles, PDL between kernels",
+              "l2": "inputs larger than L2 (W is %.0f MB > 126 MB)" % (2 * w.V * w.d / 1e6)}
+    launches = step.launches() * steps
+    del step
+    _release()
+    return {"value": value, "unit": UNIT, "steps": steps, "warmup": warmup, "ms_per_step": cyc_ms,
+            "config": config, "e2e": e2e, "gpu_launches": launches, "roofline": roof,
+            "stages_us": stages, "clocks": clk.summary()}
 
+
+def gpu_arm(args, w: syn.Workload):
+    import torch
+    rank, local_rank, world = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=torch.device("cuda", local_rank))
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    head = measure(args, w, args.steps, args.warmup, rank, world, device)
+    subs = {}
+    if world == 1 and args.sub_workloads:
+        for name in args.sub_workloads:
+            if name != w.name:
+                subs[name] = measure(args, syn.workload(name), None, args.warmup, rank, world, device)
     out = None
     if rank == 0:
         out = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded block_draft_synth; random-init weights of the workload's shapes)",
-            "config": {"workload": w.name + {"greedy": "", "sample": "+sampled-walk(T=1)",
-                                              "ctx": "+context-gated-scorer"}[args.cycle]
-                                   + ("+dynamic-conv" if args.conv == "dynamic" else ""),
-                       "blocks_per_gpu": w.B, "L": w.L, "M": w.M, "d": w.d, "V": w.V,
-                       "K": 16, "r": w.r, "conv": [w.B, w.P, w.d], "parallelism": f"dp{world} (blocks)",
-                       "cycle": args.cycle, "conv": args.conv,
-                       "launch": "eager" if args.eager else f"cuda graphs of {chunk} cycles, PDL between kernels",
-                       "l2": "inputs larger than L2 (W is %.0f MB > 126 MB)" % (2 * w.V * w.d / 1e6)},
-            "e2e": e2e,
-            "gpu_launches": step.launches() * args.steps,
-            "roofline": roof,
-            "stages_us": {**{n: 1e3 * t for n, t in zip(Step.STAGES, stage_ms)},
-                          "select_verify_share": stage_ms[2] / (ms_max / args.steps),
-                          "select_verify_added": None if sel_added_ms is None else 1e3 * sel_added_ms,
-                          "select_verify_added_share": (None if sel_added_ms is None
-                                                        else sel_added_ms / (ms_max / args.steps)),
-                          "event_pair_overhead": 1e3 * ev_ms,
-                          "raw": {n: 1e3 * t for n, t in zip(Step.STAGES, raw_ms)},
-                          "samples": len(samples["lmhead_topk"]),
-                          "note": ("durations net of the bracketing event-node pair (measured alone, 'raw' is "
-                                   "gross); select_verify_added = (LM head + selection bracketed together) - "
-                                   "(LM head bracketed alone): what the selection stage adds to a cycle when "
-                                   "its launch may overlap the LM head's end")},
-            "clocks": clk.summary(),
+            "config": head["config"], "e2e": head["e2e"], "gpu_launches": head["gpu_launches"],
+            "roofline": head["roofline"], "stages_us": head["stages_us"], "clocks": head["clocks"],
         }
+        if subs:
+            out["workloads"] = subs
+            out["workloads_note"] = ("the other workloads, each timed in this run for its own steps "
+                                     "(calibrated to about %.2f s, at least --steps), same warm-up; the headline "
+                                     "above is the largest workload" % args.sub_seconds)
         if world == 1 and not args.no_cpu_baseline:
             out["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     if world > 1:
@@ -624,13 +702,55 @@ def reference_arm(args, w: syn.Workload):
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def free_port() -> int:
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def relaunch(n: int, argv) -> int:
+    """Run this script as n ranks through torch.distributed.run on 127.0.0.1
+    (one process per GPU) and return its exit code; rank 0 prints the line."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", f"--master-port={free_port()}", os.path.abspath(__file__), *argv]
+    env = dict(os.environ, OMP_NUM_THREADS=os.environ.get("OMP_NUM_THREADS", "1"))
+    return subprocess.run(cmd, env=env).returncode
+
+
+def launch_selftest(args):
+    """Checks the N-rank launch itself on CPU (gloo): every rank joins, the
+    ranks agree on the world size, and a max over ranks reaches rank 0.  No
+    GPU, no kernel, no metric."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    rank, _, world = dist_env()
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    seen = [None] * world
+    dist.all_gather_object(seen, rank)
+    t = torch.tensor([float(rank + 1)], dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.barrier()
+    dist.destroy_process_group()
+    if rank != 0:
+        return None
+    return {"launch_selftest": True, "n_gpus": world, "ranks": seen, "max_over_ranks": float(t.item())}
+
+
 def main(argv=None):
+    argv = sys.argv[1:] if argv is None else list(argv)
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    names = [x.name for x in syn.WORKLOADS]
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=50)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
-                    choices=[x.name for x in syn.WORKLOADS])
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=names)
+    ap.add_argument("--sub-workloads", default=",".join(names),
+                    help="comma-separated workloads also timed (one GPU only) and reported under 'workloads'; "
+                         "'' for none (the headline workload is skipped here)")
+    ap.add_argument("--sub-seconds", type=float, default=0.3,
+                    help="timed seconds each extra workload aims at (at least --steps steps)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -644,11 +764,26 @@ def main(argv=None):
                     help="static base taps (the metric's path) or taps with the per-16-channel correction")
     ap.add_argument("--ref-budget-s", type=float, default=120.0,
                     help="host seconds the --impl reference run aims to take")
+    ap.add_argument("--launch-selftest", action="store_true",
+                    help="check the N-rank launch on CPU (gloo) and print the ranks seen; runs no kernel")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
+    args.sub_workloads = [x for x in args.sub_workloads.split(",") if x]
+    for x in args.sub_workloads:
+        if x not in names:
+            ap.error(f"unknown workload {x!r} in --sub-workloads")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        sys.exit(relaunch(args.gpus, argv))
+    _, _, world = dist_env()
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     w = syn.workload(args.workload)
-    if args.impl == "reference":
+    if args.launch_selftest:
+        out = launch_selftest(args)
+    elif args.impl == "reference":
         out = reference_arm(args, w)
     else:
         out = gpu_arm(args, w)

@@ -9,6 +9,8 @@ import numpy as np
 import torch
 
 from ._binding import (  # noqa: F401
+    DFLASH_ERR_BAD_INDEX,
+    DFLASH_ERR_TIMEOUT,
     DFlashError,
     K_TOP,
     LIB_PATH,

@@ -823,7 +823,15 @@ static int num_sms_current() {
   return n;
 }
 
+// Budget of every mbarrier wait of one launch.  DFLASH_TIMEOUT_NS, read at
+// every call (a positive count of nanoseconds; a process may change it
+// between calls), takes precedence over DFLASH_TIMEOUT_MS, read once per
+// process; without either the budget is 2 s.
 static unsigned long long timeout_ns_from_env() {
+  if (const char* e = std::getenv("DFLASH_TIMEOUT_NS")) {
+    const long long ns = std::atoll(e);
+    if (ns > 0) return static_cast<unsigned long long>(ns);
+  }
   static unsigned long long v = [] {
     const char* e = std::getenv("DFLASH_TIMEOUT_MS");
     long long ms = e ? std::atoll(e) : 2000;

@@ -29,9 +29,13 @@
  *     checks and launch errors.  Errors found on the device (a bounded wait
  *     that ran out, an out-of-range token index) are written with atomicCAS
  *     into `dev_status` (a device int the caller zeroes; NULL = not recorded).
- *   - Every device-side wait is bounded (default 2000 ms, environment
- *     variable DFLASH_TIMEOUT_MS overrides); a kernel that gives up records
- *     DFLASH_ERR_TIMEOUT and returns instead of hanging.
+ *   - Every device-side wait is bounded (default 2000 ms; the environment
+ *     variable DFLASH_TIMEOUT_MS, read once per process, overrides it, and
+ *     DFLASH_TIMEOUT_NS, read at every call, overrides both); a kernel that
+ *     gives up records DFLASH_ERR_TIMEOUT, drains the copies and tensor-core
+ *     operations it has in flight, releases its tensor memory and returns
+ *     instead of hanging.  The outputs of such a call are not valid; the
+ *     context stays usable for the next call.
  */
 #ifndef DFLASH_H_
 #define DFLASH_H_

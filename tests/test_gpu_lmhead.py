@@ -79,15 +79,27 @@ def test_workload_full_all_rows(wi):
     assert np.abs(lse - rlse).max() < 2e-2
 
 
+def tile_edge_rows(M, tile=128):
+    """The first and the last row of every `tile`-row token tile of M rows
+    (the last tile may be ragged): every tile of the tensor-bound schedule,
+    2-CTA pair tiles of 256 rows included, has rows in the sample."""
+    rows = []
+    for t0 in range(0, M, tile):
+        rows += [t0, min(M, t0 + tile) - 1]
+    return np.array(sorted(set(rows)))
+
+
 @pytest.mark.parametrize("wi,nrows", [(2, 24), (4, 24)])
 def test_workload_full_sampled_rows(wi, nrows):
     """Full-size tensor-bound workloads: the kernel runs on every row; the
-    oracle checks a seeded sample of rows (first, last, and random)."""
+    oracle checks the first and last row of every 128-row token tile plus a
+    seeded random sample."""
     w = syn.workload(wi)
     H, W = syn.hidden(w), syn.lm_head(w)
     lp, ix, lse = _run(H, W)
     rng = np.random.default_rng(wi)
-    rows = np.unique(np.concatenate([[0, 127, 128, w.M - 1], rng.choice(w.M, nrows, replace=False)]))
+    rows = np.unique(np.concatenate([tile_edge_rows(w.M), rng.choice(w.M, nrows, replace=False)]))
+    assert len(rows) >= 2 * ((w.M + 127) // 128)
     rlp, rix, rlse, z = oracle.lmhead_topk(H[rows], W, 16, return_logits=True)
     check_topk_rows(z, rlse, ix, lp, rows=rows)
     assert np.abs(lse[rows] - rlse).max() < 2e-2

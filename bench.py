@@ -354,6 +354,9 @@ def _chunk(steps, cap=32):
     return max(c for c in range(1, min(cap, steps) + 1) if steps % c == 0)
 
 
+# LM-head launch durations sampled inside the timed region (at least).
+LM_SAMPLES = 20
+
 # Stage breakdown: one extra graph after the timed region in which cycle k
 # brackets stage BREAKDOWN[k % 5]; every stage gets BREAKDOWN_SAMPLES samples.
 BREAKDOWN = ("event_pair", "conv2tap", "lmhead_topk", "select_verify", "lmhead_select")
@@ -415,8 +418,11 @@ def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, de
     if steps is None:
         steps = _calibrated_steps(step, args.sub_seconds, args.steps)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    # timed region: every cycle brackets its LM-head call, so the roofline's
-    # launch duration is sampled live in the timed region (one sample per step)
+    # timed region: cycles replayed from up to 64 distinct captured graphs, a
+    # few evenly spaced cycles of each bracketing their LM-head call, so the
+    # roofline's launch duration has at least LM_SAMPLES samples from the
+    # timed region (every cycle when there are no more steps than that) while
+    # most cycles keep their kernel-to-kernel launch overlap
     if args.eager:
         chunk, graphs = 1, []
         marks = [{"lmhead_topk": (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))}
@@ -424,7 +430,12 @@ def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, de
     else:
         chunk = _chunk(steps)
         n_rep = steps // chunk
-        graphs = [_graph_steps(step, chunk, lambda k: "lmhead_topk") for _ in range(min(8, n_rep))]
+        n_graphs = min(64, n_rep)
+        per_graph = min(chunk, -(-LM_SAMPLES // n_graphs))
+        spacing = chunk // per_graph
+        timed = {chunk - 1 - j * spacing for j in range(per_graph)}
+        graphs = [_graph_steps(step, chunk, lambda k: "lmhead_topk" if k in timed else None)
+                  for _ in range(n_graphs)]
         for g, _ in graphs:
             g.replay()              # one untimed replay of each captured graph
     barrier()
@@ -527,7 +538,8 @@ def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, de
     roof["launch_ms_net_of_events"] = max(1e-9, lm_ms - ev_ms)
     roof["frac_net_of_events"] = roof["frac"] * lm_ms / roof["launch_ms_net_of_events"]
     roof["timing"] = ("mean CUDA-event duration of the LM-head call (GEMM+epilogue kernel and merge kernel, "
-                      "bracketed by event nodes in every cycle of the timed graphs), over the timed region")
+                      "bracketed by event nodes in evenly spaced cycles of every timed graph: at least %d "
+                      "samples, every cycle when the run has no more steps), over the timed region" % LM_SAMPLES)
     stages = {**{n: 1e3 * stage_ms[n] for n in stage_ms},
               "select_verify_share": stage_ms["select_verify"] / cyc_ms,
               "select_verify_added": 1e3 * sel_added_ms,

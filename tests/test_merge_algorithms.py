@@ -9,7 +9,8 @@ in Python and checked against a full sort of every candidate (no GPU).
   elementwise better of a[k] and b[15-k], then four half-cleaner stages;
 - the 16-element bitonic sorting network that fills an empty list;
 - the weight-streaming tile plan: every tile width a CTA runs is one of the
-  at most four widths the host builds tensor maps for.
+  at most four widths the host builds tensor maps for, including the narrow
+  last tile of a long range.
 Ties, duplicate values, records with empty slots and few records are all
 exercised; the GPU tests check the kernels themselves."""
 import numpy as np
@@ -132,33 +133,48 @@ def test_bitonic_merge_and_sort_network(seed):
     assert _sort16(ents[:K]) == a
 
 
-def _stream_tiles(units, G, c):
+TAIL = 4   # 16-row units of the narrow last tile of a long range
+
+
+def _split(n, tail_units):
+    """stream_split: (main tiles, units per main tile, tail units)."""
+    tail = tail_units if tail_units > 0 and n >= tail_units + 16 else 0
+    m = n - tail
+    nt = -(-m // 16)
+    wu = -(-m // nt) if nt else 0
+    return nt, wu, tail
+
+
+def _stream_tiles(units, G, c, tail_units):
     """Widths (in rows) of CTA c's tiles: its balanced 16-row-unit range cut
-    into the fewest equal tiles of at most 256 rows."""
+    into the fewest equal tiles of at most 256 rows, then the narrow tail."""
     u0, u1 = c * units // G, (c + 1) * units // G
-    n = u1 - u0
-    nt = -(-n // 16)
-    wu = -(-n // nt) if nt else 0
+    nt, wu, tail = _split(u1 - u0, tail_units)
+    main_end = u1 - tail
     out = []
     for k in range(nt):
-        t0 = (u0 + k * wu) * 16
-        if t0 >= u1 * 16:
+        t0 = u0 + k * wu
+        if t0 >= main_end:
             break
-        out.append(min(wu * 16, u1 * 16 - t0))
+        out.append((min(t0 + wu, main_end) - t0) * 16)
+    if tail:
+        out.append(tail * 16)
     return out
 
 
-def _stream_widths(units, G):
-    """The widths the host enumerates (one tensor map each, at most four)."""
+def _stream_widths(units, G, tail_units):
+    """The widths the host enumerates (one tensor map each, at most four);
+    None when more than four would be needed."""
     ws = []
     u_lo = units // G
     for u in (u_lo, u_lo + 1):
         if u < 1:
             continue
-        nt = -(-u // 16)
-        wu = -(-u // nt)
-        for w in (16 * wu, 16 * (u - (nt - 1) * wu)):
+        nt, wu, tail = _split(u, tail_units)
+        for w in (16 * wu, 16 * (u - tail - (nt - 1) * wu), 16 * tail):
             if w > 0 and w not in ws:
+                if len(ws) == 4:
+                    return None
                 ws.append(w)
     return ws
 
@@ -171,11 +187,26 @@ def test_stream_tile_widths_are_enumerated(V):
     units = -(-V // 16)
     for sms in (148, 132, 8):
         G = min(units, sms)
-        ws = _stream_widths(units, G)
-        assert len(ws) <= 4
+        tail = TAIL
+        ws = _stream_widths(units, G, tail)
+        if ws is None:                 # the host drops the tail rather than need a fifth map
+            tail = 0
+            ws = _stream_widths(units, G, tail)
+        assert ws is not None and len(ws) <= 4
         covered = 0
         for c in range(G):
-            tiles = _stream_tiles(units, G, c)
+            tiles = _stream_tiles(units, G, c, tail)
             assert all(w in ws and 0 < w <= 256 for w in tiles)
             covered += sum(tiles)
+            if tail and (c + 1) * units // G - c * units // G >= tail + 16:
+                assert tiles[-1] == 16 * tail  # long ranges end with the narrow tile
         assert covered == units * 16
+
+
+def test_stream_tail_at_the_weight_streaming_workloads():
+    """qwen3-4b-bs1 and 27b-class (V = 151,936 over 148 CTAs) keep the narrow
+    64-row last tile on every CTA."""
+    units = 151936 // 16
+    assert _stream_widths(units, 148, TAIL) is not None
+    for c in range(148):
+        assert _stream_tiles(units, 148, c, TAIL)[-1] == 64

@@ -89,7 +89,6 @@ struct Params {
   int merge_halves;  // one run per unit: the two column halves merge in-kernel
   int store_only;    // plain GEMM: write z to z_dbg, no log-softmax / top-16
   int v_offset;      // added to every vocabulary index written to a record
-  int pf_ahead;      // LARGE: K stages ahead of the TMA loads whose W rows are prefetched into L2
   int w_prefetch;    // STREAM: K stages of W prefetched into L2 before the dependency wait
   int ksplit;        // plain GEMM, STREAM: CTAs per tile range, each over 1/ksplit of K
                      // (partial sums added into z_dbg, which the host zeroes first)
@@ -242,39 +241,60 @@ __device__ __forceinline__ bool get_tile(const Params& p, int k, uint32_t rank, 
 // (max, sum exp) and sorted top-16.  Called by a whole warp (one row per
 // lane): candidates that can enter a lane's list are inserted by that lane,
 // so the warp loops max over lanes of their count; an empty list (a run's
-// first chunk) is filled by sorting the chunk.
+// first chunk) is filled by sorting the chunk.  Written for instruction-level
+// parallelism: the max, the sum of exponentials and the candidate mask are
+// trees over independent values, not chains through one accumulator, and a
+// candidate's value is picked by a 4-level select tree.
 __device__ __forceinline__ void fold_chunk(TopState& st, const float (&x)[16], int vbase, int nvalid) {
-  float cmax = -INFINITY;
+  float xv[16];
 #pragma unroll
-  for (int jj = 0; jj < 16; ++jj)
-    if (jj < nvalid) cmax = fmaxf(cmax, x[jj]);
+  for (int jj = 0; jj < 16; ++jj) xv[jj] = jj < nvalid ? x[jj] : -INFINITY;
+  float t8[8], t4[4];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) t8[q] = fmaxf(xv[2 * q], xv[2 * q + 1]);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) t4[q] = fmaxf(t8[2 * q], t8[2 * q + 1]);
+  const float cmax = fmaxf(fmaxf(t4[0], t4[1]), fmaxf(t4[2], t4[3]));
   if (cmax > st.m) {
     st.s *= __expf(st.m - cmax);
     st.m = cmax;
   }
+  float e[16];
 #pragma unroll
-  for (int jj = 0; jj < 16; ++jj)
-    if (jj < nvalid) st.s += __expf(x[jj] - st.m);
+  for (int jj = 0; jj < 16; ++jj) e[jj] = __expf(xv[jj] - st.m);   // exp(-inf) = 0 for the padding
+#pragma unroll
+  for (int q = 0; q < 8; ++q) e[q] = e[2 * q] + e[2 * q + 1];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) e[q] = e[2 * q] + e[2 * q + 1];
+  st.s += (e[0] + e[1]) + (e[2] + e[3]);
   uint32_t pend = 0;
   if (nvalid == 16 && st.v[0] == -INFINITY) {
     st.assign_sorted16(x, vbase);
   } else {
+    // a candidate must beat this list's 16th entry
+    const float thr = st.v[KTOP - 1];
+    uint32_t b4[4];
 #pragma unroll
-    for (int jj = 0; jj < 16; ++jj)
-      if (jj < nvalid && x[jj] > st.v[KTOP - 1]) pend |= 1u << jj;
+    for (int q = 0; q < 4; ++q)
+      b4[q] = (xv[4 * q] > thr ? 1u : 0u) | (xv[4 * q + 1] > thr ? 2u : 0u) | (xv[4 * q + 2] > thr ? 4u : 0u) |
+              (xv[4 * q + 3] > thr ? 8u : 0u);
+    pend = (b4[0] | (b4[1] << 4)) | ((b4[2] << 8) | (b4[3] << 12));
   }
   while (__any_sync(0xffffffffu, pend != 0)) {
     if (pend) {
       const int jj = __ffs(pend) - 1;
       pend &= pend - 1;
-      float xv = x[0];
+      float s8[8], s4[4], s2[2];
 #pragma unroll
-      for (int q = 1; q < 16; ++q) xv = jj == q ? x[q] : xv;
-      st.insert_scan(xv, vbase + jj);
+      for (int q = 0; q < 8; ++q) s8[q] = (jj & 1) ? x[2 * q + 1] : x[2 * q];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) s4[q] = (jj & 2) ? s8[2 * q + 1] : s8[2 * q];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) s2[q] = (jj & 4) ? s4[2 * q + 1] : s4[2 * q];
+      st.insert_scan((jj & 8) ? s2[1] : s2[0], vbase + jj);
     }
   }
 }
-
 
 // First K stage of this CTA's share of K (split only for the plain GEMM in
 // STREAM mode: CTAs [ks*G, (ks+1)*G) take the ks-th of ksplit slices).
@@ -385,12 +405,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         else
           tma_load_2d_hint(dst, m, fb, c0, c1, pol);
       };
-      Tile t, tn;
+      Tile t;
       for (int k = 0; ok && get_tile<MODE, PAIR>(p, k, rank, t); ++k) {
-        // LARGE: W rows pf_ahead stages ahead are pulled into L2 as each stage
-        // is loaded (this tile's later stages, then the next tile's first),
-        // so a load that misses L2 waits for HBM less often
-        const bool has_next = MODE == MODE_LARGE && p.pf_ahead > 0 && get_tile<MODE, PAIR>(p, k + 1, rank, tn);
         // bytes landing on the leader's barrier per stage (both CTAs of a pair)
         const int b_rows_here = MODE == MODE_STREAM ? t.n_cols : p.b_rows;
         const uint32_t tx = static_cast<uint32_t>((PAIR ? 2 : 1) * (p.a_box + b_rows_here) * BK * 2);
@@ -412,13 +428,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             else if (b_rows_here == p.b_widths[3]) mb = &tm_w3;
           }
           load(b_dst, mb, fb, kc * BK, t.b_row, pol_w);
-          if (MODE == MODE_LARGE && p.pf_ahead > 0) {
-            const int ka = kc + p.pf_ahead;
-            if (ka < kc1)
-              tma_prefetch_l2_2d(&tm_b, ka * BK, t.b_row);
-            else if (has_next && ka - kc1 < kc1)
-              tma_prefetch_l2_2d(&tm_b, (ka - kc1) * BK, tn.b_row);
-          }
           issued_mask |= 1u << s;
           issued_par = (issued_par & ~(1u << s)) | (ph << s);
           if (++s == p.stages) { s = 0; ph ^= 1u; }
@@ -621,376 +630,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tmem_dealloc_pair(tmem_base, p.tmem_cols);
     else
       tmem_dealloc(tmem_base, p.tmem_cols);
-  }
-}
-
-// ------------------------------------------------- wide pair tiles --------
-// Tensor-bound orientation on a cluster of two CTAs, one work step = 256
-// token rows x up to 512 vocabulary rows ("wide tile"): per K stage each CTA
-// stages 128 token rows of H (16 KB) and its 128-row halves of two 256-row
-// vocabulary sub-tiles (32 KB); the leader issues two tcgen05.mma.cta_group::2
-// of M = 256, N = 256 that share the token operand.  Per multiply-add this
-// moves a quarter fewer bytes from L2 into shared memory than a 256 x 256
-// step (48 KB per 4.2M multiply-adds per CTA instead of 32 KB per 2.1M).
-// The accumulator takes all 512 TMEM columns, in two halves with their own
-// "free" barriers: the epilogue folds half 0, frees it, folds half 1, frees
-// it; the MMA issuer starts the next tile's half-0 products as soon as half 0
-// is free and holds the stages (up to the whole ring) whose half-1 products
-// must wait for half 1, so the epilogue is mostly hidden behind the products.
-// At the end of each job the two column-halves of a row (the two epilogue
-// warps of a lane quarter) merge in a dedicated shared-memory area and one
-// partial record per (row, job) is written.
-constexpr int WIDE_SUB = 2;                          // N = 256 sub-tiles per wide tile
-constexpr int WIDE_A_STAGE = A_ROWS * BK * 2;        // 16 KB
-constexpr int WIDE_B_SUB = (TILE_N / 2) * BK * 2;    // 16 KB: one CTA's half of a sub-tile
-constexpr int WIDE_B_STAGE = WIDE_SUB * WIDE_B_SUB;  // 32 KB
-constexpr int XCH_FLOATS = 36;                       // exchange record per row
-
-struct WideLayout {
-  uint32_t a, b, xch, bars, misc, total;
-};
-
-__host__ __device__ inline WideLayout wide_layout(int stages) {
-  WideLayout s;
-  s.a = 0;
-  s.b = s.a + stages * WIDE_A_STAGE;
-  s.xch = s.b + stages * WIDE_B_STAGE;
-  s.bars = s.xch + A_ROWS * XCH_FLOATS * 4;
-  s.misc = s.bars + (2 * stages + 4) * 8;
-  s.total = s.misc + 16;
-  return s;
-}
-
-struct WideTile {
-  int a_row;   // first token row of this CTA's half of the token tile
-  int b_row;   // first W row this CTA loads for sub-tile 0 (sub-tile 1: + 256)
-  int n_sub;   // 1 or 2 sub-tiles of 256 vocabulary rows
-  int v0;      // vocabulary index of accumulator column 0
-  int slot;    // record slot of the job
-  bool first, last;
-};
-
-// The k-th wide step of this CTA pair; false past the end.  RUNS: unit u owns
-// token tile u % m_tiles over vocabulary range u / m_tiles of nr (in 256-row
-// tiles, walked two at a time).  BLOCKS: jobs (token tile, block of R
-// vocabulary tiles), block-major, dealt round-robin to the units.
-__device__ __forceinline__ bool get_wide_tile(const Params& p, int k, uint32_t rank, WideTile& t) {
-  const int u = static_cast<int>(blockIdx.x >> 1);
-  const int units = static_cast<int>(gridDim.x >> 1);
-  int mt, vt, hi;
-  if (p.sched == SCHED_RUNS) {
-    mt = u % p.m_tiles;
-    const int r = u / p.m_tiles;
-    const int lo = static_cast<int>(static_cast<long long>(r) * p.v_tiles / p.nr);
-    hi = static_cast<int>(static_cast<long long>(r + 1) * p.v_tiles / p.nr);
-    vt = lo + WIDE_SUB * k;
-    if (vt >= hi) return false;
-    t.slot = r;
-    t.first = k == 0;
-    t.last = vt + WIDE_SUB >= hi;
-  } else {
-    const long long jobs = static_cast<long long>(p.m_tiles) * p.n_vblocks;
-    long long job = u;
-    int kk = k;
-    for (;;) {
-      if (job >= jobs) return false;
-      const int vb = static_cast<int>(job / p.m_tiles);
-      const int lo = vb * p.R;
-      hi = min(lo + p.R, p.v_tiles);
-      const int nsteps = (hi - lo + WIDE_SUB - 1) / WIDE_SUB;
-      if (kk < nsteps) {
-        mt = static_cast<int>(job - static_cast<long long>(vb) * p.m_tiles);
-        vt = lo + WIDE_SUB * kk;
-        t.slot = vb;
-        t.first = kk == 0;
-        t.last = kk == nsteps - 1;
-        break;
-      }
-      kk -= nsteps;
-      job += units;
-    }
-  }
-  t.n_sub = min(WIDE_SUB, hi - vt);
-  t.a_row = mt * 2 * A_ROWS + static_cast<int>(rank) * A_ROWS;
-  t.b_row = vt * TILE_N + static_cast<int>(rank) * (TILE_N / 2);
-  t.v0 = vt * TILE_N;
-  return true;
-}
-
-__global__ void __launch_bounds__(NUM_THREADS, 1)
-    lmhead_wide_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                       const Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  const WideLayout L = wide_layout(p.stages);
-  const int S = p.stages;
-  const uint32_t sbase = smem_addr(smem);
-  const uint32_t bar0 = sbase + L.bars;
-  auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
-  const uint32_t tfull_bar = bar0 + 8u * (2 * S);
-  auto tempty_bar = [&](int h) { return bar0 + 8u * (2 * S + 1 + h); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * S + 3);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 4);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const bool leader = rank == 0;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
-    }
-    mbar_init(tfull_bar, 1);
-    mbar_init(tempty_bar(0), 2 * EPI_THREADS);
-    mbar_init(tempty_bar(1), 2 * EPI_THREADS);
-    mbar_init(drain_bar, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tm_a);
-    prefetch_tmap(&tm_b);
-  }
-  if (warp == 1) tmem_alloc_pair(smem_addr(tmem_slot), p.tmem_cols);
-  tc_fence_before();
-  __syncthreads();
-  __syncwarp();
-  cluster_sync_all();  // both CTAs' barriers exist before any remote signal
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-  pdl_wait();
-  const uint64_t deadline = globaltimer_ns() + p.timeout_ns;
-
-  if (warp == 0) {
-    // ------------------------------------------------------ TMA producer --
-    if (lane == 0) {
-      const uint64_t pol_keep = l2_policy_evict_last();
-      const uint64_t pol_w = l2_policy_evict_normal();
-      int s = 0;
-      uint32_t ph = 0;
-      uint32_t issued_mask = 0, issued_par = 0;
-      bool ok = true;
-      WideTile t;
-      for (int k = 0; ok && get_wide_tile(p, k, rank, t); ++k) {
-        // bytes landing on the leader's barrier per stage (both CTAs)
-        const uint32_t tx = static_cast<uint32_t>(2 * (WIDE_A_STAGE + t.n_sub * WIDE_B_SUB));
-        for (int kc = 0; kc < p.num_kc; ++kc) {
-          if (!mbar_wait(empty_bar(s), ph ^ 1u, deadline, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          const uint32_t fb = full_bar(s);
-          const uint32_t fb_leader = mapa_shared(fb, 0);
-          if (leader) mbar_arrive_expect_tx(fb, tx);
-          tma_load_2d_pair(sbase + L.a + s * WIDE_A_STAGE, &tm_a, fb_leader, kc * BK, t.a_row, pol_keep);
-          const uint32_t b_dst = sbase + L.b + s * WIDE_B_STAGE;
-          for (int h = 0; h < t.n_sub; ++h)
-            tma_load_2d_pair(b_dst + h * WIDE_B_SUB, &tm_b, fb_leader, kc * BK, t.b_row + h * TILE_N, pol_w);
-          issued_mask |= 1u << s;
-          issued_par = (issued_par & ~(1u << s)) | (ph << s);
-          if (++s == S) { s = 0; ph ^= 1u; }
-        }
-      }
-      if (!ok) {
-        // Do not leave with copies in flight (see lmhead_kernel): the leader
-        // waits, bounded, for the last load into every stage; the other CTA's
-        // loads complete on the leader's barriers, so it waits a fixed time.
-        const uint64_t dl = globaltimer_ns() + 50000000ull;
-        if (leader) {
-          for (int q = 0; q < S; ++q) {
-            if (!(issued_mask >> q & 1u)) continue;
-            const uint32_t par = (issued_par >> q) & 1u;
-            while (!mbar_try_wait(full_bar(q), par) && globaltimer_ns() < dl) {
-            }
-          }
-        } else {
-          const uint64_t t_end = globaltimer_ns() + 200000ull;
-          while (globaltimer_ns() < t_end) {
-          }
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------ MMA issuer ----
-    if (lane == 0 && leader) {
-      const uint32_t idesc = umma_idesc_bf16_f32(2 * A_ROWS, TILE_N);
-      int s = 0;
-      uint32_t ph = 0;
-      uint32_t tph = 0;
-      bool ok = true;
-      auto products = [&](int stage, int h, bool first_stage) {
-        const uint64_t adesc = umma_desc_sw128(sbase + L.a + stage * WIDE_A_STAGE);
-        const uint64_t bdesc = umma_desc_sw128(sbase + L.b + stage * WIDE_B_STAGE + h * WIDE_B_SUB);
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(h * TILE_N);
-#pragma unroll
-        for (int kk = 0; kk < BK / UMMA_K; ++kk)
-          umma_bf16_pair(d_tmem, adesc + 2ull * kk, bdesc + 2ull * kk, idesc, (first_stage && kk == 0) ? 0u : 1u);
-      };
-      WideTile t;
-      for (int k = 0; ok && get_wide_tile(p, k, rank, t); ++k) {
-        // half 0 must be free (the previous tile's epilogue folded it)
-        if (!mbar_wait(tempty_bar(0), tph ^ 1u, deadline, abort_flag, p.status)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        bool h1_free = false;
-        int npend = 0, ps = s;   // stages whose half-1 products are still to issue, from ring index ps
-        for (int kc = 0; kc < p.num_kc; ++kc) {
-          if (!mbar_wait(full_bar(s), ph, deadline, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          products(s, 0, kc == 0);
-          if (t.n_sub == 2) {
-            if (!h1_free) {
-              h1_free = mbar_test_wait(tempty_bar(1), tph ^ 1u);   // never suspends the issuer
-              if (!h1_free && npend + 1 == S) {
-                // every stage of the ring is held: wait for half 1
-                if (!mbar_wait(tempty_bar(1), tph ^ 1u, deadline, abort_flag, p.status)) {
-                  ok = false;
-                  break;
-                }
-                h1_free = true;
-              }
-              if (h1_free) tc_fence_after();
-            }
-            if (h1_free) {
-              for (int q = 0; q < npend; ++q) {
-                const int st_q = (ps + q) % S;
-                products(st_q, 1, kc - npend + q == 0);
-                umma_commit_pair_multicast(empty_bar(st_q), 0x3);
-              }
-              npend = 0;
-              products(s, 1, kc == 0);
-              umma_commit_pair_multicast(empty_bar(s), 0x3);
-            } else {
-              if (npend == 0) ps = s;
-              ++npend;
-            }
-          } else {
-            umma_commit_pair_multicast(empty_bar(s), 0x3);
-          }
-          if (++s == S) { s = 0; ph ^= 1u; }
-        }
-        if (!ok) break;
-        if (!h1_free) {
-          // a narrow tile still consumes half 1's phase; a wide one issues
-          // the half-1 products it held back
-          if (!mbar_wait(tempty_bar(1), tph ^ 1u, deadline, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          for (int q = 0; q < npend; ++q) {
-            const int st_q = (ps + q) % S;
-            products(st_q, 1, p.num_kc - npend + q == 0);
-            umma_commit_pair_multicast(empty_bar(st_q), 0x3);
-          }
-        }
-        umma_commit_pair_multicast(tfull_bar, 0x3);
-        tph ^= 1u;
-      }
-      // Every MMA this thread issued has completed before TMEM is released.
-      umma_commit_pair(drain_bar);
-      const uint64_t dl = globaltimer_ns() + 50000000ull;
-      while (!mbar_try_wait(drain_bar, 0) && globaltimer_ns() < dl) {
-      }
-    }
-  } else {
-    // ------------------------------------------------------ epilogue ------
-    const int ew = warp - 2;                  // 0..7
-    const int quarter = warp & 3;             // TMEM lanes this warp may access
-    const int half = ew >> 2;                 // which half of each sub-tile's columns
-    const int trow = quarter * 32 + lane;     // accumulator row held by this thread
-    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    float* xs = reinterpret_cast<float*>(smem + L.xch) + trow * XCH_FLOATS;
-    TopState st;
-    st.reset();
-    uint32_t tph = 0;
-    WideTile t;
-    for (int k = 0; get_wide_tile(p, k, rank, t); ++k) {
-      int ok = 0;
-      if (lane == 0) ok = mbar_wait(tfull_bar, tph, deadline, abort_flag, p.status) ? 1 : 0;
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      // All epilogue warps leave together or go on together: the job-end
-      // exchange below synchronises pairs of them.
-      if (!named_barrier_and(5, EPI_THREADS, ok != 0)) break;
-      tc_fence_after();
-      if (t.first) st.reset();
-      const int row = t.a_row + trow;
-      const bool active = t.a_row + quarter * 32 < p.M;  // any of this warp's rows real
-      for (int h = 0; h < WIDE_SUB; ++h) {
-        if (active && h < t.n_sub) {
-          const uint32_t taddr = tmem_base + static_cast<uint32_t>(h * TILE_N) + lane_off;
-          for (int ch = half * 8; ch < half * 8 + 8; ++ch) {
-            const int c0 = ch * 16;
-            const int vbase = t.v0 + h * TILE_N + c0;
-            if (vbase >= p.V) break;
-            float x[16];
-            tmem_ld16(taddr + c0, x);
-            tmem_ld_wait();
-            const int nvalid = min(16, p.V - vbase);
-            fold_chunk(st, x, vbase, nvalid);
-            if (p.z_dbg && row < p.M) {
-#pragma unroll
-              for (int jj = 0; jj < 16; ++jj)
-                if (jj < nvalid) p.z_dbg[static_cast<size_t>(row) * p.V + vbase + jj] = x[jj];
-            }
-          }
-        }
-        // release this half of the accumulator (the leader's barrier)
-        tc_fence_before();
-        if (leader)
-          mbar_arrive(tempty_bar(h));
-        else
-          mbar_arrive_cluster(mapa_shared(tempty_bar(h), 0));
-      }
-      tph ^= 1u;
-      if (t.last) {
-        // the job's two column-halves of each row merge into one record
-        if (half == 1) {
-          xs[0] = st.m;
-          xs[1] = st.s;
-#pragma unroll
-          for (int q = 0; q < KTOP; ++q) {
-            xs[2 + q] = st.v[q];
-            xs[18 + q] = __int_as_float(st.i[q]);
-          }
-        }
-        named_barrier_sync(1 + quarter, 64);
-        if (half == 0 && row < p.M) {
-          float ov[KTOP];
-          int oi[KTOP];
-#pragma unroll
-          for (int q = 0; q < KTOP; ++q) {
-            ov[q] = xs[2 + q];
-            oi[q] = __float_as_int(xs[18 + q]);
-          }
-          st.merge_lse(xs[0], xs[1]);
-          st.merge_bitonic(ov, oi);
-          store_record(p.part + static_cast<size_t>(row) * p.P + t.slot, st, p.v_offset);
-        }
-        named_barrier_sync(1 + quarter, 64);   // the area is free for the next job
-      }
-    }
-  }
-
-  pdl_trigger();
-  tc_fence_before();
-  __syncthreads();
-  __syncwarp();
-  cluster_sync_all();  // the pair's MMAs and remote arrivals are done
-  if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc_pair(tmem_base, p.tmem_cols);
   }
 }
 
@@ -1377,103 +1016,13 @@ static int max_pair_clusters() {
   return n;
 }
 
-static cudaError_t set_smem_attr_wide() {
-  static std::once_flag once;
-  static cudaError_t err = cudaSuccess;
-  std::call_once(once, [] {
-    err = cudaFuncSetAttribute(lmhead_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BUDGET + 2048);
-  });
-  return err;
-}
-
-// Clusters of two of the wide kernel that can be resident at once.
-static int max_wide_clusters() {
-  static std::once_flag once;
-  static int n = 0;
-  std::call_once(once, [] {
-    if (set_smem_attr_wide() != cudaSuccess) return;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2);
-    cfg.blockDim = dim3(NUM_THREADS);
-    cfg.dynamicSmemBytes = SMEM_BUDGET + 1024;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int c = 0;
-    if (cudaOccupancyMaxActiveClusters(&c, lmhead_wide_kernel, &cfg) == cudaSuccess) n = c;
-    cudaGetLastError();
-  });
-  return n;
-}
-
-// Wide pair tiles are used for the tensor-bound orientation only with
-// DFLASH_WIDE=1 (read at every call): they move a quarter fewer bytes from L2
-// per product but leave the epilogue less room to hide (single-buffered
-// accumulator), which costs more than it saves with the present epilogue.
-static bool wide_allowed() {
-  const char* e = std::getenv("DFLASH_WIDE");
-  return e != nullptr && e[0] == '1';
-}
-
 struct Plan {
   int mode;
   bool pair;
-  bool wide;   // LARGE on pairs with wide (256 x 512) tiles: lmhead_wide_kernel
   int grid;
   Params p;
   size_t smem;
 };
-
-// L2 bytes the concurrently running jobs of a wide BLOCKS schedule keep
-// reading (W rows of the vocabulary blocks in flight) above which W would be
-// fetched from HBM more than once.
-constexpr double WIDE_W_WINDOW_BYTES = 48.0 * 1024 * 1024;
-
-// Schedule of the wide orientation over `units` pairs: RUNS, or BLOCKS(R)
-// with R an even number of 256-row vocabulary tiles, chosen by the tiles on
-// the busiest unit (a job restart charged as 0.15 tile), among the BLOCKS
-// whose W window stays within WIDE_W_WINDOW_BYTES.  Returns the units used.
-static int plan_wide_schedule(Params& p, int units) {
-  const double restart = 0.15;
-  double best = 1e30;
-  int used = 1;
-  int nr = units / p.m_tiles;
-  if (nr > p.v_tiles) nr = p.v_tiles;
-  if (nr >= 1) {
-    const long long t_run = (p.v_tiles + nr - 1) / nr;
-    best = t_run * (1.0 + restart / t_run);
-    p.sched = SCHED_RUNS;
-    p.nr = nr;
-    p.R = 0;
-    p.n_vblocks = 0;
-    p.P = nr;
-    used = nr * p.m_tiles;
-  }
-  const double tile_bytes = static_cast<double>(TILE_N) * p.d * 2;
-  for (int R = 2; R <= 64; R *= 2) {
-    const int nvb = (p.v_tiles + R - 1) / R;
-    const long long jobs = static_cast<long long>(p.m_tiles) * nvb;
-    const int u = static_cast<int>(jobs < units ? jobs : units);
-    const double window = (static_cast<double>(u) / p.m_tiles + 1.0) * R * tile_bytes;
-    if (R > 2 && window > WIDE_W_WINDOW_BYTES) break;
-    const long long t_blk = ((jobs + u - 1) / u) * R;
-    const double c = t_blk * (1.0 + restart / R);
-    if (c < best) {
-      best = c;
-      p.sched = SCHED_BLOCKS;
-      p.R = R;
-      p.n_vblocks = nvb;
-      p.nr = 0;
-      p.P = nvb;
-      used = u;
-    }
-  }
-  return used;
-}
 
 // Deepest ring of `per_stage` bytes that fits the shared-memory budget.
 static int fit_stages(Params& p, int cap) {
@@ -1495,11 +1044,10 @@ static int stream_tail_units() {
   return v < 0 ? 0 : (v > 8 ? 8 : v);
 }
 
-static bool make_plan(int M, int V, int d, int sms, Plan& pl, bool allow_wide = true, bool store_only = false) {
+static bool make_plan(int M, int V, int d, int sms, Plan& pl, bool store_only = false) {
   if (M < 1 || V < 16 || d < 8 || d % 8 != 0 || sms < 1) return false;
   Params& p = pl.p;
   p = Params{};
-  pl.wide = false;
   p.M = M;
   p.V = V;
   p.d = d;
@@ -1549,27 +1097,6 @@ static bool make_plan(int M, int V, int d, int sms, Plan& pl, bool allow_wide = 
       p.tail_units = 0;
     }
     if (fit_stages(p, 12) < 2) return false;
-  } else if (allow_wide && pair_allowed() && wide_allowed() && max_wide_clusters() >= 1) {
-    pl.mode = MODE_LARGE;
-    pl.pair = true;
-    pl.wide = true;
-    p.a_box = A_ROWS;
-    p.a_stage_bytes = WIDE_A_STAGE;
-    p.b_rows = TILE_N / 2;
-    p.b_stage_bytes = WIDE_B_STAGE;
-    p.m_tiles = (M + 2 * A_ROWS - 1) / (2 * A_ROWS);
-    p.v_tiles = (V + TILE_N - 1) / TILE_N;
-    const int clusters = max_wide_clusters();
-    const int units = clusters < sms / 2 ? clusters : sms / 2;
-    if (units < 1) return false;
-    const int used = plan_wide_schedule(p, units);
-    pl.grid = 2 * used;
-    p.stages = 0;
-    for (int st = 2; st <= 8; ++st)
-      if (wide_layout(st).total + 1024 <= static_cast<uint32_t>(SMEM_BUDGET)) p.stages = st;
-    if (p.stages < 2) return false;
-    pl.smem = wide_layout(p.stages).total + 1024;
-    return true;
   } else {
     pl.mode = MODE_LARGE;
     const int clusters = pair_allowed() ? max_pair_clusters<MODE_LARGE>() : 0;
@@ -1621,7 +1148,7 @@ static bool make_plan(int M, int V, int d, int sms, Plan& pl, bool allow_wide = 
       }
     }
     pl.grid = pl.pair ? 2 * used : used;
-    if (fit_stages(p, env_int("DFLASH_MAX_STAGES", 8, 2, 8)) < 2) return false;
+    if (fit_stages(p, 8) < 2) return false;
   }
   pl.smem = smem_layout(p).total + 1024;
   return true;
@@ -1637,12 +1164,6 @@ static cudaError_t launch_main(const Plan& pl, const CUtensorMap& ta, const CUte
   if (e != cudaSuccess) return e;
   return launch_kernel_cluster(lmhead_kernel<MODE, PAIR>, dim3(pl.grid), dim3(NUM_THREADS), pl.smem, st,
                                PAIR ? 2 : 1, ta, tb[0], tb[1], tb[2], tb[3], pl.p);
-}
-
-static cudaError_t launch_wide(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, cudaStream_t st) {
-  const cudaError_t e = set_smem_attr_wide();
-  if (e != cudaSuccess) return e;
-  return launch_kernel_cluster(lmhead_wide_kernel, dim3(pl.grid), dim3(NUM_THREADS), pl.smem, st, 2, ta, tb, pl.p);
 }
 
 static cudaError_t launch_merge(const Partial* part, int M, int Pr, int nrank, float* topk_logp,
@@ -1670,7 +1191,7 @@ static int launch(const dflash_bf16* H, const dflash_bf16* W, int M, int V, int 
       (reinterpret_cast<uintptr_t>(ws) & 255) || (store_only && (reinterpret_cast<uintptr_t>(z_dbg) & 15)))
     return DFLASH_ERR_INVALID_ARG;
   Plan pl;
-  if (!make_plan(M, V, d, num_sms_current(), pl, !store_only, store_only)) return DFLASH_ERR_INVALID_ARG;
+  if (!make_plan(M, V, d, num_sms_current(), pl, store_only)) return DFLASH_ERR_INVALID_ARG;
   if (!store_only && ws_bytes < part_bytes(pl)) return DFLASH_ERR_WORKSPACE;
   Params& p = pl.p;
   p.part = static_cast<Partial*>(ws);
@@ -1692,7 +1213,6 @@ static int launch(const dflash_bf16* H, const dflash_bf16* W, int M, int V, int 
   p.z_dbg = z_dbg;
   p.status = dev_status;
   p.timeout_ns = timeout_ns_from_env();
-  p.pf_ahead = env_int("DFLASH_PF_AHEAD", 0, 0, 64);
   p.w_prefetch = env_int("DFLASH_W_PREFETCH", 8, 0, 64);
 
   // W maps: the full tile box, then (STREAM) one box per other tile width
@@ -1713,8 +1233,6 @@ static int launch(const dflash_bf16* H, const dflash_bf16* W, int M, int V, int 
     return DFLASH_ERR_CUDA;
   if (pl.mode == MODE_STREAM)
     e = launch_main<MODE_STREAM, false>(pl, ta, tb, st);
-  else if (pl.wide)
-    e = launch_wide(pl, ta, tb[0], st);
   else
     e = pl.pair ? launch_main<MODE_LARGE, true>(pl, ta, tb, st) : launch_main<MODE_LARGE, false>(pl, ta, tb, st);
   if (e != cudaSuccess) return DFLASH_ERR_CUDA;

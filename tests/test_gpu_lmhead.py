@@ -116,45 +116,3 @@ def test_repeat_calls_identical():
     b = _run(H, W)
     for x, y in zip(a, b):
         np.testing.assert_array_equal(x, y)
-
-
-@pytest.fixture
-def wide_tiles(monkeypatch):
-    """The tensor-bound orientation's wide-tile kernel (two N = 256 products
-    per K stage sharing the token operand), which the library runs only when
-    DFLASH_WIDE=1 (read at every call)."""
-    monkeypatch.setenv("DFLASH_WIDE", "1")
-
-
-LARGE_SHAPES = [(129, 3000, 128), (200, 2600, 192), (300, 517, 64), (448, 4000, 256), (700, 9000, 320)]
-
-
-@pytest.mark.parametrize("M,V,d", LARGE_SHAPES)
-def test_wide_logits_within_bound(M, V, d, wide_tiles):
-    import block_draft_selection_b200 as bds
-    H, W = _inputs(M, V, d, 3 * M + V)
-    z = bds.dflash_lmhead_logits_debug(dev_bf16(H), dev_bf16(W))
-    torch.cuda.synchronize()
-    z = z.cpu().numpy().astype(np.float64)
-    err = np.abs(z - oracle.logits(H, W))
-    assert (err <= logits_bound(H, W)).all(), err.max()
-
-
-@pytest.mark.parametrize("M,V,d", LARGE_SHAPES)
-def test_wide_topk(M, V, d, wide_tiles):
-    H, W = _inputs(M, V, d, 5 * M + V)
-    lp, ix, lse = _run(H, W)
-    rlp, rix, rlse, z = oracle.lmhead_topk(H, W, 16, return_logits=True)
-    check_topk_rows(z, rlse, ix, lp)
-    assert np.abs(lse - rlse).max() < 2e-2
-
-
-def test_wide_workload_batched(wide_tiles):
-    """qwen3-4b-batched through the wide kernel: the first and last row of
-    every 128-row token tile plus a random sample against the oracle."""
-    w = syn.workload(2)
-    H, W = syn.hidden(w), syn.lm_head(w)
-    lp, ix, lse = _run(H, W)
-    rows = np.unique(np.concatenate([tile_edge_rows(w.M), np.random.default_rng(9).choice(w.M, 16, replace=False)]))
-    rlp, rix, rlse, z = oracle.lmhead_topk(H[rows], W, 16, return_logits=True)
-    check_topk_rows(z, rlse, ix, lp, rows=rows)

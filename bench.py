@@ -505,8 +505,9 @@ def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, de
         h2d, d2h = cyc.io_bytes()
         e2e = {"value": aggregate(w.B, world, e_ms, steps), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-               "path": "DraftCycle.run(): pinned H2D + conv + LM head + select/verify + D2H (with the status word), "
-                       "host sync"}
+               "path": "DraftCycle.run(): one graph launch per step: pinned H2D of H + targets + zeroed status, "
+                       "LM head, select/verify, D2H of status + results; beside it on a second stream H2D of the "
+                       "conv input, conv, D2H of its output; host sync"}
         del cyc
     else:
         e2e = {"value": None, "unit": UNIT, "h2d_bytes_per_step": None, "d2h_bytes_per_step": None,

@@ -135,11 +135,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with acquire at cluster scope: what another CTA of the cluster
+// wrote before its release-arrive on this barrier is visible afterwards.
+__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Store a 32-bit value into another CTA's shared memory (a shared::cluster
+// address from mapa).
+__device__ __forceinline__ void st_shared_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
 // Wait for the phase with the given parity to complete, at most until
 // `deadline` (globaltimer ns) or until *abort becomes nonzero.  Returns false
-// (and records a timeout) when it gives up.
+// (and records a timeout) when it gives up.  A nonzero `peer_abort` (the
+// shared::cluster address of the other CTA's abort flag in a pair) is set
+// too, so both CTAs of a pair stop together.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t deadline,
-                                          volatile int* abort, int* status) {
+                                          volatile int* abort, int* status, uint32_t peer_abort = 0) {
   uint32_t spins = 0;
   while (!mbar_try_wait(bar, parity)) {
     if ((++spins & 63u) == 0) {
@@ -147,11 +169,18 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
       if (globaltimer_ns() > deadline) {
         set_status(status, DFLASH_ERR_TIMEOUT);
         *abort = 1;
+        if (peer_abort != 0) st_shared_cluster_u32(peer_abort, 1u);
         return false;
       }
     }
   }
   return true;
+}
+
+// Count `bytes` as arrived on the barrier's current phase without a copy
+// (the transaction count drops as if they had landed).
+__device__ __forceinline__ void mbar_complete_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
 
 // ---------------------------------------------------------------- TMA -------

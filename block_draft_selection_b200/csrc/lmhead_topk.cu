@@ -142,7 +142,7 @@ __host__ __device__ inline SmemLayout smem_layout(const Params& p) {
   uint32_t b_min = (p.stages - 1) * p.a_stage_bytes + MMA_A_SPAN;
   if (s.b < b_min) s.b = (b_min + 1023) & ~1023u;
   s.bars = s.b + p.stages * p.b_stage_bytes;
-  s.misc = s.bars + (2 * p.stages + 5) * 8;
+  s.misc = s.bars + (2 * p.stages + 6) * 8;
   s.total = s.misc + 16;
   return s;
 }
@@ -321,13 +321,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * p.stages + b); };
   auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * p.stages + 2 + b); };
   const uint32_t drain_bar = bar0 + 8u * (2 * p.stages + 4);
+  // pair: the other CTA hands its count of stage loads to the leader here
+  const uint32_t handover_bar = bar0 + 8u * (2 * p.stages + 5);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 4);
+  volatile int* peer_issued = reinterpret_cast<volatile int*>(smem + L.misc + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
   const bool leader = rank == 0;
+  // a wait that gives up in one CTA of a pair stops the other one too
+  const uint32_t peer_abort = PAIR ? mapa_shared(smem_addr(const_cast<int*>(abort_flag)), rank ^ 1u) : 0u;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
@@ -339,7 +344,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(tempty_bar(b), PAIR ? 2 * EPI_THREADS : EPI_THREADS);
     }
     mbar_init(drain_bar, 1);
+    mbar_init(handover_bar, 1);
     *abort_flag = 0;
+    *peer_issued = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -387,6 +394,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int kc0 = kc0_of(p);
   const int kc1 = (ks + 1) * p.num_kc / p.ksplit;
 
+  int issued = 0;   // producer: stage loads issued, in ring order (load k went to stage k % stages)
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
@@ -397,7 +405,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint64_t pol_w = MODE == MODE_STREAM ? pol_stream : pol_normal;
       int s = 0;
       uint32_t ph = 0;
-      uint32_t issued_mask = 0, issued_par = 0;
       bool ok = true;
       auto load = [&](uint32_t dst, const CUtensorMap* m, uint32_t fb, int c0, int c1, uint64_t pol) {
         if (PAIR)
@@ -411,7 +418,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int b_rows_here = MODE == MODE_STREAM ? t.n_cols : p.b_rows;
         const uint32_t tx = static_cast<uint32_t>((PAIR ? 2 : 1) * (p.a_box + b_rows_here) * BK * 2);
         for (int kc = kc0; kc < kc1; ++kc) {
-          if (!mbar_wait(empty_bar(s), ph ^ 1u, deadline, abort_flag, p.status)) {
+          if (!mbar_wait(empty_bar(s), ph ^ 1u, deadline, abort_flag, p.status, peer_abort)) {
             ok = false;
             break;
           }
@@ -428,29 +435,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             else if (b_rows_here == p.b_widths[3]) mb = &tm_w3;
           }
           load(b_dst, mb, fb, kc * BK, t.b_row, pol_w);
-          issued_mask |= 1u << s;
-          issued_par = (issued_par & ~(1u << s)) | (ph << s);
+          ++issued;
           if (++s == p.stages) { s = 0; ph ^= 1u; }
         }
       }
-      if (!ok) {
-        // Do not leave with copies in flight.  A leader (or a single CTA)
-        // waits, bounded, for the last load into every stage to land; in a
-        // pair the other CTA's loads complete on the leader's barriers, so it
-        // waits a fixed, bounded time instead.
-        const uint64_t dl = globaltimer_ns() + 50000000ull;
-        if (leader) {
-          for (int q = 0; q < p.stages; ++q) {
-            if (!(issued_mask >> q & 1u)) continue;
-            const uint32_t par = (issued_par >> q) & 1u;
-            while (!mbar_try_wait(full_bar(q), par) && globaltimer_ns() < dl) {
-            }
-          }
-        } else {
-          const uint64_t t_end = globaltimer_ns() + 200000ull;
-          while (globaltimer_ns() < t_end) {
-          }
-        }
+      // pair: the other CTA hands the leader its count of loads (always: it
+      // cannot know whether the leader will need it; see the drain below)
+      if (PAIR && !leader) {
+        st_shared_cluster_u32(mapa_shared(smem_addr(const_cast<int*>(peer_issued)), 0), static_cast<uint32_t>(issued));
+        mbar_arrive_cluster(mapa_shared(handover_bar, 0));   // release: the count is visible first
       }
     }
   } else if (warp == 1) {
@@ -470,14 +463,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       Tile t;
       for (int k = 0; ok && get_tile<MODE, PAIR>(p, k, rank, t); ++k) {
         const uint32_t idesc = umma_idesc_bf16_f32(PAIR ? 2 * A_ROWS : A_ROWS, t.n_cols);
-        if (!mbar_wait(tempty_bar(tb), tph ^ 1u, deadline, abort_flag, p.status)) {
+        if (!mbar_wait(tempty_bar(tb), tph ^ 1u, deadline, abort_flag, p.status, peer_abort)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(tb * TILE_N);
         for (int kc = kc0; kc < kc1; ++kc) {
-          if (!mbar_wait(full_bar(s), ph, deadline, abort_flag, p.status)) {
+          if (!mbar_wait(full_bar(s), ph, deadline, abort_flag, p.status, peer_abort)) {
             ok = false;
             break;
           }
@@ -525,7 +518,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     Tile t;
     for (int k = 0; get_tile<MODE, PAIR>(p, k, rank, t); ++k) {
       int ok = 0;
-      if (lane == 0) ok = mbar_wait(tfull_bar(tb), tph, deadline, abort_flag, p.status) ? 1 : 0;
+      if (lane == 0) ok = mbar_wait(tfull_bar(tb), tph, deadline, abort_flag, p.status, peer_abort) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
@@ -622,7 +615,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   __syncwarp();
-  if (PAIR) cluster_sync_all();  // the pair's MMAs and remote arrivals are done
+  if (PAIR) cluster_sync_all();  // every role of both CTAs is done: abort flags and counts are final
+  if (warp == 0 && lane == 0 && leader && *abort_flag != 0) {
+    // Never leave with copies in flight: after giving up, the loads that
+    // were issued but never consumed must be seen to land before the CTA
+    // (and, in a pair, the other CTA) may exit.  Every load of a pair
+    // completes on the leader's barriers, so the leader drains both CTAs'
+    // loads.  Both CTAs fill the stages in the same order and one runs at
+    // most a ring ahead of the other (a stage is refilled only after both
+    // its loads were consumed), so the two counts say which stage loads
+    // only one CTA issued: for a load only the leader issued, the other
+    // CTA's bytes will never come and are counted as arrived (complete_tx);
+    // for one only the other CTA issued, the leader's arrival is made with
+    // that CTA's bytes alone (arrive.expect_tx).  The last phase of every
+    // stage then completes exactly when its last copy has landed.
+    const uint64_t dl = globaltimer_ns() + 50000000ull;
+    int n_all = issued;
+    if (PAIR && mbar_try_wait_acq_cluster(handover_bar, 0)) {   // arrived before the cluster barrier
+      const int n_peer = *peer_issued;
+      const uint32_t peer_tx = static_cast<uint32_t>((p.a_box + p.b_rows) * BK * 2);
+      const int k_lo = min(issued, n_peer), k_hi = max(issued, n_peer);
+      for (int k = k_lo; k < k_hi; ++k) {
+        if (issued > n_peer)
+          mbar_complete_tx(full_bar(k % p.stages), peer_tx);
+        else
+          mbar_arrive_expect_tx(full_bar(k % p.stages), peer_tx);
+      }
+      n_all = k_hi;
+    }
+    for (int q = 0; q < p.stages && q < n_all; ++q) {
+      const int k_last = q + ((n_all - 1 - q) / p.stages) * p.stages;   // last load into stage q
+      const uint32_t par = static_cast<uint32_t>(k_last / p.stages) & 1u;
+      while (!mbar_try_wait(full_bar(q), par) && globaltimer_ns() < dl) {
+      }
+    }
+  }
+  if (PAIR) {
+    __syncwarp();
+    cluster_sync_all();  // the other CTA stays resident until the leader's drain is done
+  }
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
@@ -1308,9 +1339,11 @@ extern "C" int dflash_lmhead_topk_merge(const void* records, int M, int P, int n
 //
 // Host code cannot use `g_static_scratch` as a pointer (its host-side name is
 // only a stand-in for the device symbol), so the device address is looked up
-// with cudaGetSymbolAddress once per device, with that device current, on the
-// first call made while it is current.  That first call on a device should
-// therefore happen before any stream capture begins.
+// with cudaGetSymbolAddress once per device and CUDA context, with that device
+// current, on the first call made in that context (again after a
+// cudaDeviceReset, which gives the device a new context and the array a new
+// address).  That first call should therefore happen before any stream
+// capture begins.
 //
 // Every call shares the one array: calls that can overlap on the GPU (other
 // streams, other host threads on the same device) race on it and must be
@@ -1326,16 +1359,40 @@ namespace lm {
 constexpr int kMaxDevices = 64;
 static std::mutex g_static_mu;
 static void* g_static_ptr[kMaxDevices] = {};
+static void* g_static_ctx[kMaxDevices] = {};
 
-// Device address of g_static_scratch on the current device (looked up once).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// The calling thread's current CUDA context (nullptr if it cannot be read).
+static void* current_context() {
+  static CtxGetCurrentFn fn = [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<CtxGetCurrentFn>(nullptr);
+    return reinterpret_cast<CtxGetCurrentFn>(ptr);
+  }();
+  CUcontext c = nullptr;
+  if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// Device address of g_static_scratch on the current device.  It is looked
+// up once per (device, context): a context created after cudaDeviceReset
+// (or after the primary context was released) holds the array at a new
+// address, so the cached one is refreshed whenever the current context is
+// not the one it was read in.
 static int static_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DFLASH_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_static_mu);
-  if (g_static_ptr[dev] == nullptr) {
+  void* ctx = current_context();
+  if (g_static_ptr[dev] == nullptr || ctx == nullptr || ctx != g_static_ctx[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return DFLASH_ERR_CUDA;
     g_static_ptr[dev] = p;
+    g_static_ctx[dev] = current_context();  // the lookup may have just made the primary context current
   }
   *out = g_static_ptr[dev];
   return DFLASH_OK;

@@ -13,9 +13,10 @@
 //
 // Two kernels:
 //   1. row statistics: CTA (row, slice) reduces 8192 logits of one row to
-//      (m, s): y = z*c in fp64 with c = log2(e) / T, m = max y, s = sum of
-//      exp2(y - m) (fp32 exponential of the fp64 difference, fp64 sum) --
-//      also the slice's probability mass once the row is merged;
+//      (m, s) with c = log2(e) / T: m = c * max z, s = sum of
+//      exp2((z - max z) * c) (fp32 exponentials added in pairs in fp32, the
+//      pair sums in fp64) -- also the slice's probability mass once the row
+//      is merged;
 //   2. one CTA of 1024 threads per block: merges its L+1 rows' statistics,
 //      tests the L drafts (one lane each), picks the residual's slice from
 //      the slice masses (corrected at the 16 candidates), then scans that
@@ -93,8 +94,16 @@ __global__ void __launch_bounds__(T1) row_stats_kernel(const float* __restrict__
   double m = static_cast<double>(xm) * c;  // c > 0: the max of z*c is at the max of z
   double s = 0.0;
   if (xm != -INFINITY) {
+    // exp2((x - xm) * c) in fp32; neighbouring pairs added in fp32 (one
+    // rounding, at most 2^-24 relative, below exp2f's own error), the pair
+    // sums widened and added in fp64.  x - xm is exact wherever x >= xm / 2
+    // (the terms that carry the sum) and otherwise off by at most 2^-24 of a
+    // difference whose term is tiny; the product adds one rounding relative
+    // to the exponent, i.e. |y| * 2^-24 * ln 2 relative to the term.
+    const float cf = static_cast<float>(c);
 #pragma unroll
-    for (int j = 0; j < EPT1; ++j) s += static_cast<double>(exp2f(static_cast<float>(x[j] * c - m)));
+    for (int j = 0; j < EPT1; j += 2)
+      s += static_cast<double>(exp2f((x[j] - xm) * cf) + exp2f((x[j + 1] - xm) * cf));   // padding: 0
   }
 #pragma unroll
   for (int off = 16; off; off >>= 1) {

@@ -7,11 +7,15 @@ inputs from pinned host buffers to the device, runs the cycle and copies its
 results back, all captured once into a CUDA graph so a step costs one graph
 launch on the host.  Weights (W, E, M, conv taps) stay on the device.
 
-The step's inputs, a status word and its results live in one device buffer
-(each tensor at a 256-byte-aligned offset), mirrored by a pinned host buffer
-for the inputs and one for the results: a step moves its inputs (and a zero
-status word) with one host-to-device copy and the status word and its results
-with one device-to-host copy, and `run()` raises if the status is nonzero.
+A step has two lanes.  The selection lane's inputs (hidden states, target
+tokens), a status word and its results live in one device buffer (each
+tensor at a 256-byte-aligned offset), mirrored by a pinned host buffer for
+the inputs and one for the results: one host-to-device copy moves the inputs
+and a zero status word, one device-to-host copy the status word and the
+results, and `run()` raises if the status is nonzero.  The conv does not feed
+the LM head, so its lane (one copy of its inputs in, the conv, one copy of its
+output out) runs on a second stream inside the same graph, overlapping the
+LM head; the step ends when both lanes have.
 """
 from __future__ import annotations
 
@@ -75,10 +79,10 @@ class DraftCycle:
         V, d = W.shape
         M = B * L
         e = lambda shape, dt: torch.empty(shape, dtype=dt, device=dev)
-        ins = [("H", (M, d), torch.bfloat16), ("x", (B, P, d), torch.bfloat16), ("prev", (B, d), torch.bfloat16),
-               ("target", (B, L + 1), torch.int32)]
+        # selection lane: hidden states and targets in; status and the path's results out
+        ins = [("H", (M, d), torch.bfloat16), ("target", (B, L + 1), torch.int32)]
         outs = [("path_tok", (B, L), torch.int32), ("accept_len", (B,), torch.int32),
-                ("next_token", (B,), torch.int32), ("y", (B, P, d), torch.bfloat16)]
+                ("next_token", (B,), torch.int32)]
         # one device buffer (inputs | status | results) and pinned host twins
         # of its input span and its result span
         offs, in_end, out_begin, end = io_layout(ins, outs)
@@ -89,14 +93,23 @@ class DraftCycle:
         self._din, self._dout = self._dbuf[:in_end], self._dbuf[out_begin:]
         self._hin = torch.zeros(in_end, dtype=torch.uint8, pin_memory=True)    # its status word stays 0
         self._hout = torch.zeros(end - out_begin, dtype=torch.uint8, pin_memory=True)
-        self.host_in = _views(self._hin, offs, in_names[:-1])
-        self.host_out = _views(self._hout, offs, out_names, base=out_begin)
-        self.H, self.x, self.prev, self.target = dv["H"], dv["x"], dv["prev"], dv["target"]
-        self.tok, self.acc, self.nxt, self.y = dv["path_tok"], dv["accept_len"], dv["next_token"], dv["y"]
+        # conv lane: the conv's input and previous-position rows in, its output out
+        cins = [("x", (B, P, d), torch.bfloat16), ("prev", (B, d), torch.bfloat16)]
+        couts = [("y", (B, P, d), torch.bfloat16)]
+        self._cdin, cdin = _arena(cins, dev)
+        self._cdout, cdout = _arena(couts, dev)
+        self._chin, chin = _arena(cins, "cpu", pinned=True)
+        self._chout, chout = _arena(couts, "cpu", pinned=True)
+        self.host_in = {**_views(self._hin, offs, in_names[:-1]), **chin}
+        self.host_out = {**_views(self._hout, offs, out_names, base=out_begin), **chout}
+        self.H, self.target = dv["H"], dv["target"]
+        self.x, self.prev, self.y = cdin["x"], cdin["prev"], cdout["y"]
+        self.tok, self.acc, self.nxt = dv["path_tok"], dv["accept_len"], dv["next_token"]
         self.lp, self.ix, self.lse = e((M, 16), torch.float32), e((M, 16), torch.int32), e((M,), torch.float32)
         self.slot, self.score = e((B, L), torch.int32), e((B,), torch.float32)
         self.status = dv["status"]
         self.ws = b.workspace(M, V, d, dev)
+        self._side = torch.cuda.Stream(device=dev)
         self._graph = None
         if use_graph:
             self._capture()
@@ -104,6 +117,9 @@ class DraftCycle:
     def kernels(self):
         """Enqueue the cycle's kernels on the current stream (device buffers)."""
         b.dflash_conv2tap(self.x, self.a0, self.a1, self.prev, y=self.y)
+        self.selection_kernels()
+
+    def selection_kernels(self):
         b.dflash_lmhead_topk(self.H, self.W, topk_logp=self.lp, topk_idx=self.ix, lse=self.lse, ws=self.ws,
                              dev_status=self.status)
         b.dflash_select_verify(self.lp, self.ix, self.E, self.Msel, self.target, self.B, self.L,
@@ -111,20 +127,31 @@ class DraftCycle:
                                accept_len=self.acc, next_token=self.nxt, dev_status=self.status)
 
     def _step(self):
-        self._din.copy_(self._hin, non_blocking=True)      # one host-to-device copy
-        self.kernels()
-        self._hout.copy_(self._dout, non_blocking=True)    # one device-to-host copy
+        """The conv does not feed the LM head, so its lane (copy in, conv,
+        copy out) runs on a side stream alongside the selection lane (copy
+        in, LM head, selection + verification, copy out); the step ends when
+        both have."""
+        main = torch.cuda.current_stream()
+        self._side.wait_stream(main)
+        with torch.cuda.stream(self._side):
+            self._cdin.copy_(self._chin, non_blocking=True)
+            b.dflash_conv2tap(self.x, self.a0, self.a1, self.prev, y=self.y)
+            self._chout.copy_(self._cdout, non_blocking=True)
+        self._din.copy_(self._hin, non_blocking=True)
+        self.selection_kernels()
+        self._hout.copy_(self._dout, non_blocking=True)
+        main.wait_stream(self._side)
 
     def _capture(self):
-        side = torch.cuda.Stream()
-        side.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(side):
+        cap = torch.cuda.Stream()
+        cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cap):
             self._step()                      # warm-up outside capture (first-call set-up)
-        side.synchronize()
+        cap.synchronize()
         self._graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(self._graph, stream=side):
+        with torch.cuda.graph(self._graph, stream=cap):
             self._step()
-        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.current_stream().wait_stream(cap)
 
     def run(self):
         """One step: host inputs (self.host_in) -> device -> cycle -> host
@@ -142,6 +169,6 @@ class DraftCycle:
         return self.host_out
 
     def io_bytes(self):
-        """Bytes a step copies host-to-device and device-to-host (the arenas,
-        alignment padding included)."""
-        return int(self._hin.numel()), int(self._hout.numel())
+        """Bytes a step copies host-to-device and device-to-host (both lanes'
+        arenas, alignment padding included)."""
+        return (int(self._hin.numel() + self._chin.numel()), int(self._hout.numel() + self._chout.numel()))

@@ -155,7 +155,9 @@ int dflash_lmhead_topk(const dflash_bf16* H, const dflash_bf16* W, int M, int V,
  * (M <= 128 at V = 151,936 fits; large-M shapes generally do not).
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current, so make that first call
- * before any stream capture.  Calls share the array: calls that may overlap
+ * before any stream capture.  The address is kept per device and CUDA
+ * context: after cudaDeviceReset (a new context, the array at a new address)
+ * the next call looks it up again.  Calls share the array: calls that may overlap
  * on the GPU (different streams or threads on one device) race and must be
  * serialised by the caller.  The call allocates no memory.
  */

@@ -235,6 +235,8 @@ class Step:
         self.tok, self.slot = e((w.B, w.L), torch.int32), e((w.B, w.L), torch.int32)
         self.score, self.acc, self.nxt = e(w.B, torch.float32), e(w.B, torch.int32), e(w.B, torch.int32)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.side = torch.cuda.Stream(device=dev)     # timing events hang off the kernel chain here
+        self.marked = False
         self.cycle, self.conv = cycle, conv
         if conv == "dynamic":
             self.Wc = bds.bf16_tensor(syn.conv_correction(w), dev)
@@ -272,21 +274,46 @@ class Step:
             self.cycle, self.LAUNCHES_PER_STEP)
         return n + (1 if self.conv == "dynamic" else 0)   # the dynamic conv adds its correction GEMM
 
-    def run(self, marks=None):
+    def mark(self, ev):
+        """Record `ev` when everything enqueued so far on the current stream
+        has completed, on a side stream: the event hangs off the kernel chain
+        instead of sitting in it, so consecutive kernels keep their
+        programmatic (early) launch.  Inside graph capture the side stream
+        must be joined back before the capture ends (see join_marks)."""
+        import torch
+        cur = torch.cuda.current_stream()
+        self.side.wait_stream(cur)
+        with torch.cuda.stream(self.side):
+            ev.record()
+        self.marked = True
+
+    def join_marks(self):
+        import torch
+        if self.marked:
+            torch.cuda.current_stream().wait_stream(self.side)
+            self.marked = False
+
+    def run(self, marks=None, side=False):
         """One cycle.  `marks`: optional {stage name: (event, event)} recorded
-        around that stage's call; "event_pair" brackets nothing (the cost of
-        the two event nodes) and "lmhead_select" brackets the LM head and the
-        selection stage together."""
+        around that stage's call.  side=False: the events sit in the kernel
+        chain (the bracketed stage's first kernel then starts only after the
+        start event, without the programmatic early launch); side=True: they
+        hang off the chain on a side branch (see mark), so the kernels keep
+        their early launch -- accurate for long stages, while two side
+        events are never less than a few microseconds apart.  "event_pair"
+        brackets nothing (the cost of the two event nodes) and
+        "lmhead_select" brackets the LM head and the selection together."""
         bds = self.bds
         marks = marks or {}
+        put = self.mark if side else (lambda e: e.record())
 
         def stage(name, fn):
             ev = marks.get(name)
             if ev:
-                ev[0].record()
+                put(ev[0])
             fn()
             if ev:
-                ev[1].record()
+                put(ev[1])
 
         stage("event_pair", lambda: None)    # calibration: two event nodes, nothing between
         if self.conv == "dynamic":
@@ -296,7 +323,7 @@ class Step:
             stage("conv2tap", lambda: bds.dflash_conv2tap(self.x, self.a0, self.a1, self.prev, y=self.y))
         span = marks.get("lmhead_select")
         if span:
-            span[0].record()
+            put(span[0])
         stage("lmhead_topk", lambda: bds.dflash_lmhead_topk(
             self.H, self.W, topk_logp=self.lp, topk_idx=self.ix, lse=self.lse, ws=self.ws, dev_status=self.status))
         if self.cycle == "sample":
@@ -324,13 +351,14 @@ class Step:
                 path_slot=self.slot, path_score=self.score, accept_len=self.acc, next_token=self.nxt,
                 dev_status=self.status))
         if span:
-            span[1].record()
+            put(span[1])
 
 
-def _graph_steps(step, n_steps, plan):
+def _graph_steps(step, n_steps, plan, side=False):
     """Capture n_steps cycles into one CUDA graph.  plan(k) names the stage
     whose call cycle k brackets with a pair of external timing events (event
-    nodes), or None.  Returns (graph, [(stage name, (start, end))])."""
+    nodes; in the kernel chain, or on a side branch with side=True), or
+    None.  Returns (graph, [(stage name, (start, end))])."""
     import torch
     ev = lambda: (torch.cuda.Event(enable_timing=True, external=True),
                   torch.cuda.Event(enable_timing=True, external=True))
@@ -343,7 +371,8 @@ def _graph_steps(step, n_steps, plan):
     side.synchronize()
     with torch.cuda.graph(g, stream=side):
         for k in range(n_steps):
-            step.run(marks[k])
+            step.run(marks[k], side=side)
+        step.join_marks()          # a timing side branch rejoins once, at the end
     torch.cuda.current_stream().wait_stream(side)
     torch.cuda.synchronize()
     return g, [(name, pair) for m in marks if m for name, pair in m.items()]
@@ -437,7 +466,7 @@ def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, de
         # middle cycle (the last cycle of a graph measured about 10 us slower
         # at qwen3-4b-bs1 than the same stage anywhere else)
         timed = {spacing // 2 + j * spacing for j in range(per_graph)}
-        graphs = [_graph_steps(step, chunk, lambda k: "lmhead_topk" if k in timed else None)
+        graphs = [_graph_steps(step, chunk, lambda k: "lmhead_topk" if k in timed else None, side=True)
                   for _ in range(n_graphs)]
         for g, _ in graphs:
             g.replay()              # one untimed replay of each captured graph
@@ -446,7 +475,8 @@ def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, de
         t0.record()
         if args.eager:
             for k in range(steps):
-                step.run(marks[k])
+                step.run(marks[k], side=True)
+            step.join_marks()
         else:
             for rep in range(n_rep):
                 graphs[rep % len(graphs)][0].replay()
@@ -479,6 +509,7 @@ def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, de
     del sg, sm
     med = lambda n: statistics.median(samples[n])
     ev_ms = med("event_pair")
+    # in-chain brackets: net of the cost of the two event nodes (measured alone)
     stage_ms = {n: max(0.0, med(n) - ev_ms) for n in ("conv2tap", "lmhead_topk", "select_verify")}
     # what the selection stage adds to a cycle: (LM head + selection bracketed
     # together) - (LM head bracketed alone); both gross, the event cost cancels
@@ -539,11 +570,11 @@ def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, de
     roof["algorithmic_per_launch"] = alg_bytes if roof["bound"] == "hbm" else alg_flops
     roof["launch_ms"] = lm_ms
     roof["launch_ms_samples"] = _summ(lm_samples)
-    roof["launch_ms_net_of_events"] = max(1e-9, lm_ms - ev_ms)
-    roof["frac_net_of_events"] = roof["frac"] * lm_ms / roof["launch_ms_net_of_events"]
-    roof["timing"] = ("mean CUDA-event duration of the LM-head call (GEMM+epilogue kernel and merge kernel, "
-                      "bracketed by event nodes in evenly spaced cycles of every timed graph: at least %d "
-                      "samples, every cycle when the run has no more steps), over the timed region" % LM_SAMPLES)
+    roof["timing"] = ("mean CUDA-event duration of the LM-head call (GEMM+epilogue kernel and merge kernel), from "
+                      "the completion of the kernel before it to the completion of its merge kernel; events recorded "
+                      "on a side branch of the graph so the kernels keep their programmatic launch; evenly spaced "
+                      "cycles of every timed graph: at least %d samples (every cycle when the run has no more "
+                      "steps), over the timed region" % LM_SAMPLES)
     stages = {**{n: 1e3 * stage_ms[n] for n in stage_ms},
               "select_verify_share": stage_ms["select_verify"] / cyc_ms,
               "select_verify_added": 1e3 * sel_added_ms,
@@ -553,10 +584,12 @@ def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, de
               "raw_us": {n: {k: (1e3 * v if k != "n" else v) for k, v in _summ(samples[n]).items()}
                          for n in BREAKDOWN},
               "note": ("medians over one extra graph after the timed region whose cycle k brackets stage "
-                       "k mod 5 (%d samples per stage), net of the bracketing event-node pair (measured alone); "
+                       "k mod 5 (%d samples per stage) with event nodes in the kernel chain, net of the two "
+                       "event nodes (measured alone): a bracketed stage's first kernel starts only after the "
+                       "start event, so its time includes that kernel's launch latency; "
                        "select_verify_added = (LM head + selection bracketed together) - (LM head bracketed "
-                       "alone): what the selection stage adds to a cycle when its launch may overlap the LM "
-                       "head's end" % BREAKDOWN_SAMPLES)}
+                       "alone): what the selection adds when its launch overlaps the LM head's end, as in "
+                       "unbracketed cycles" % BREAKDOWN_SAMPLES)}
     config = {"workload": w.name + {"greedy": "", "sample": "+sampled-walk(T=1)",
                                     "ctx": "+context-gated-scorer"}[args.cycle]
                           + ("+dynamic-conv" if args.conv == "dynamic" else ""),

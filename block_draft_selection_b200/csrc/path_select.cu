@@ -9,9 +9,9 @@
 // Walk: delta_0 = 0, delta_{i+1}[k] = max_j delta_i[j] + S_i[j,k] (ties: lowest
 // j), end at argmax_k delta_{L-1}[k] (ties: lowest k), then backtrack.
 //
-// One thread-block cluster of Q CTAs (256 threads each) per block; Q = 1 when
-// there are enough blocks to fill the GPU, else up to 8 so that a block's
-// pair scoring spreads over Q SMs:
+// One thread-block cluster of Q CTAs per block; Q = 1 (one CTA of 512
+// threads) when there are enough blocks to fill the GPU, else up to 8 CTAs of
+// 256 threads so that a block's pair scoring spreads over Q SMs:
 //   1. each CTA gathers the E rows of the positions it scores and the matrix
 //      M into shared memory (bf16, rows padded by 16 bytes so 16-byte loads
 //      of 8 neighbouring rows hit distinct banks);
@@ -34,6 +34,7 @@
 // of its E row, log-probability 0), so the first pair table is
 //   S_a[k] = lp[0,k] + (e_anchor M) . e_{c_0k}
 // and internal position p >= 1 is drafted position p - 1.
+#include <cstdlib>
 #include <mutex>
 
 #include <cooperative_groups.h>
@@ -44,7 +45,8 @@
 namespace dflash {
 namespace sel {
 
-constexpr int THREADS = 256;
+constexpr int THREADS = 512;         // launch bound: 512 per CTA when Q = 1
+constexpr int THREADS_CLUSTER = 256; // per CTA of a cluster (Q > 1)
 constexpr int MAX_CLUSTER = 8;
 constexpr int KC = 16;
 constexpr int U_BUDGET = 48 * 1024;
@@ -186,15 +188,23 @@ __global__ void __launch_bounds__(THREADS) path_select_kernel(
     const uint4* Mg = reinterpret_cast<const uint4*>(Msel);
     if (use_mma) {
       // transposed, rows padded to rp: column t of M is row t here, so the
-      // tensor-core B fragments are 32-bit loads without bank conflicts
-      for (int q = tid; q < r * r8; q += nthr) {
-        const int srow = q / r8;
-        const int c8 = q - srow * r8;
-        const uint4 v = __ldg(Mg + q);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      // tensor-core B fragments are 32-bit loads without bank conflicts.  A
+      // warp moves one 8-column group of 32 consecutive source rows: lane l
+      // reads row 32*blk + l and its 16-bit stores land in neighbouring
+      // halfwords of each destination row (no bank conflicts, where lanes
+      // walking the columns of one row would all hit one bank).
+      const int lane = tid & 31, nwarp = nthr >> 5;
+      const int nblk = (r + 31) / 32;
+      for (int item = tid >> 5; item < r8 * nblk; item += nwarp) {
+        const int c8 = item % r8;
+        const int srow = (item / r8) * 32 + lane;
+        if (srow < r) {
+          const uint4 v = __ldg(Mg + static_cast<size_t>(srow) * r8 + c8);
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          Ms[static_cast<size_t>(c8 * 8 + e) * lo.rp + srow] = static_cast<uint16_t>(w[e >> 1] >> (16 * (e & 1)));
+          for (int e = 0; e < 8; ++e)
+            Ms[static_cast<size_t>(c8 * 8 + e) * lo.rp + srow] = static_cast<uint16_t>(w[e >> 1] >> (16 * (e & 1)));
+        }
       }
     } else {
       uint4* Mv = reinterpret_cast<uint4*>(Ms);
@@ -293,21 +303,23 @@ __global__ void __launch_bounds__(THREADS) path_select_kernel(
       const int i = q_rank + Q * (m0 + ii);
       const float* ur = Us + static_cast<size_t>(ii * KC + j) * lo.up;
       const uint16_t* er = Es + static_cast<size_t>((i + 1) * KC + k) * lo.rp;
-      float acc = 0.f;
+      // four independent accumulators (not one chain of r dependent FMAs)
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll 4
       for (int t = 0; t < r; t += 8) {
         const float4 u0 = *reinterpret_cast<const float4*>(ur + t);
         const float4 u1 = *reinterpret_cast<const float4*>(ur + t + 4);
         const uint4 ev = *reinterpret_cast<const uint4*>(er + t);
-        acc = fmaf(u0.x, bf_lo(ev.x), acc);
-        acc = fmaf(u0.y, bf_hi(ev.x), acc);
-        acc = fmaf(u0.z, bf_lo(ev.y), acc);
-        acc = fmaf(u0.w, bf_hi(ev.y), acc);
-        acc = fmaf(u1.x, bf_lo(ev.z), acc);
-        acc = fmaf(u1.y, bf_hi(ev.z), acc);
-        acc = fmaf(u1.z, bf_lo(ev.w), acc);
-        acc = fmaf(u1.w, bf_hi(ev.w), acc);
+        a0 = fmaf(u0.x, bf_lo(ev.x), a0);
+        a1 = fmaf(u0.y, bf_hi(ev.x), a1);
+        a2 = fmaf(u0.z, bf_lo(ev.y), a2);
+        a3 = fmaf(u0.w, bf_hi(ev.y), a3);
+        a0 = fmaf(u1.x, bf_lo(ev.z), a0);
+        a1 = fmaf(u1.y, bf_hi(ev.z), a1);
+        a2 = fmaf(u1.z, bf_lo(ev.w), a2);
+        a3 = fmaf(u1.w, bf_hi(ev.w), a3);
       }
+      const float acc = (a0 + a1) + (a2 + a3);
       const float sc = (lps[i * KC + j] + lps[(i + 1) * KC + k]) + acc;
       S_out[(i * KC + j) * KC + k] = sc;
       if (WALK == WALK_VITERBI && pair_dbg) pair_dbg[((static_cast<size_t>(b) * npos + i) * KC + j) * KC + k] = sc;
@@ -361,13 +373,20 @@ static int launch(const float* topk_logp, const int32_t* topk_idx, const dflash_
   int sms = 148, dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // DFLASH_SELECT_Q (read at every call) caps Q (1: always one CTA per block)
+  int q_cap = MAX_CLUSTER;
+  if (const char* ev = std::getenv("DFLASH_SELECT_Q")) {
+    const int v = std::atoi(ev);
+    if (v >= 1 && v <= MAX_CLUSTER) q_cap = v;
+  }
   int Q = 1;
   if (B * 2 < sms && npairs > 1) {
-    Q = npairs < MAX_CLUSTER ? npairs : MAX_CLUSTER;
+    Q = npairs < q_cap ? npairs : q_cap;
     while (Q > 1 && static_cast<long long>(B) * Q > sms) --Q;
   }
   const cudaError_t e = launch_kernel_cluster(
-      path_select_kernel<WALK>, dim3(B * Q), dim3(THREADS), lo.total, static_cast<cudaStream_t>(stream), Q,
+      path_select_kernel<WALK>, dim3(B * Q), dim3(Q > 1 ? THREADS_CLUSTER : THREADS), lo.total,
+      static_cast<cudaStream_t>(stream), Q,
       topk_logp, topk_idx, reinterpret_cast<const uint16_t*>(E), reinterpret_cast<const uint16_t*>(Msel), L, r, V,
       path_tok, path_slot, path_score, pair_scores_dbg, dev_status, target, accept_len, next_token, Q, wa);
   return e == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;

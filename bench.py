@@ -575,21 +575,25 @@ def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, de
                       "on a side branch of the graph so the kernels keep their programmatic launch; evenly spaced "
                       "cycles of every timed graph: at least %d samples (every cycle when the run has no more "
                       "steps), over the timed region" % LM_SAMPLES)
-    stages = {**{n: 1e3 * stage_ms[n] for n in stage_ms},
-              "select_verify_share": stage_ms["select_verify"] / cyc_ms,
-              "select_verify_added": 1e3 * sel_added_ms,
-              "select_verify_added_share": sel_added_ms / cyc_ms,
+    # the selection's cost in the cycle: (LM head + selection) - LM head, two
+    # long brackets (a bracket around the short selection alone is not
+    # reliable: its kernel may launch before the start event is recorded)
+    stages = {"conv2tap": 1e3 * stage_ms["conv2tap"], "lmhead_topk": 1e3 * stage_ms["lmhead_topk"],
+              "select_verify": 1e3 * sel_added_ms,
+              "select_verify_share": sel_added_ms / cyc_ms,
+              "select_verify_bracketed_alone": 1e3 * stage_ms["select_verify"],
               "event_pair_overhead": 1e3 * ev_ms,
               "samples": {n: len(samples[n]) for n in BREAKDOWN},
               "raw_us": {n: {k: (1e3 * v if k != "n" else v) for k, v in _summ(samples[n]).items()}
                          for n in BREAKDOWN},
               "note": ("medians over one extra graph after the timed region whose cycle k brackets stage "
                        "k mod 5 (%d samples per stage) with event nodes in the kernel chain, net of the two "
-                       "event nodes (measured alone): a bracketed stage's first kernel starts only after the "
-                       "start event, so its time includes that kernel's launch latency; "
-                       "select_verify_added = (LM head + selection bracketed together) - (LM head bracketed "
-                       "alone): what the selection adds when its launch overlaps the LM head's end, as in "
-                       "unbracketed cycles" % BREAKDOWN_SAMPLES)}
+                       "event nodes (measured alone); select_verify = (LM head + selection bracketed "
+                       "together) - (LM head bracketed alone): what selection and verification add to a "
+                       "cycle; select_verify_bracketed_alone is the selection bracketed by itself, for "
+                       "reference only (a few-microsecond bracket is not reliable: the bracketed kernel can "
+                       "be launched before the start event is recorded, so its samples split between its "
+                       "full time and a fraction of it)" % BREAKDOWN_SAMPLES)}
     config = {"workload": w.name + {"greedy": "", "sample": "+sampled-walk(T=1)",
                                     "ctx": "+context-gated-scorer"}[args.cycle]
                           + ("+dynamic-conv" if args.conv == "dynamic" else ""),

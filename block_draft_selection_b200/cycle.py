@@ -130,14 +130,16 @@ class DraftCycle:
         """The conv does not feed the LM head, so its lane (copy in, conv,
         copy out) runs on a side stream alongside the selection lane (copy
         in, LM head, selection + verification, copy out); the step ends when
-        both have."""
+        both have.  The conv lane starts once the selection lane's input copy
+        is done, so the copy that gates the LM head has the host link to
+        itself and the conv lane's copies overlap the LM head."""
         main = torch.cuda.current_stream()
+        self._din.copy_(self._hin, non_blocking=True)
         self._side.wait_stream(main)
         with torch.cuda.stream(self._side):
             self._cdin.copy_(self._chin, non_blocking=True)
             b.dflash_conv2tap(self.x, self.a0, self.a1, self.prev, y=self.y)
             self._chout.copy_(self._cdout, non_blocking=True)
-        self._din.copy_(self._hin, non_blocking=True)
         self.selection_kernels()
         self._hout.copy_(self._dout, non_blocking=True)
         main.wait_stream(self._side)

@@ -138,6 +138,7 @@ __global__ void __launch_bounds__(T2) reject_kernel(
   __shared__ double row_m[MAX_L + 1];
   __shared__ double row_s[MAX_L + 1];
   __shared__ double mass[MAX_SLICES];
+  __shared__ Part parts_s[MAX_L + 1][MAX_SLICES];   // every row's slice statistics, read once
   __shared__ int cand_s[KC];
   __shared__ float q_s[KC];
   __shared__ double wsum[T2 / 32];
@@ -198,6 +199,7 @@ __global__ void __launch_bounds__(T2) reject_kernel(
     double s = 0.0;
     for (int j = lane; j < S; j += 32) {
       const Part p = part[(row0 + warp) * S + j];
+      parts_s[warp][j] = p;
       merge_ms(m, s, p.m, p.s);
     }
 #pragma unroll
@@ -231,7 +233,7 @@ __global__ void __launch_bounds__(T2) reject_kernel(
   const int n = sh_n;
   const size_t R = row0 + n;  // the row the next token is drawn from
   const double mx = row_m[n];
-  const double sR = row_s[n];
+  const double inv_sR = 1.0 / row_s[n];   // one division; each probability below is a product
   const float* zr = z + R * V;
 
   // C. slice masses of p_R, minus q_n at the candidates (rejection only)
@@ -240,13 +242,13 @@ __global__ void __launch_bounds__(T2) reject_kernel(
     q_s[tid] = n < L ? pc_q[n][tid] : 0.f;
   }
   for (int j = tid; j < S; j += T2) {
-    const Part p = part[R * S + j];
-    mass[j] = p.m == -INFINITY ? 0.0 : exp2(p.m - mx) * p.s / sR;
+    const Part p = parts_s[n][j];
+    mass[j] = p.m == -INFINITY ? 0.0 : exp2(p.m - mx) * p.s * inv_sR;
   }
   __syncthreads();
   if (tid < KC && cand_s[tid] >= 0) {
     const int v = cand_s[tid];
-    const double pv = exp2(static_cast<double>(pc_z[n][tid]) * c - mx) / sR;
+    const double pv = exp2(static_cast<double>(pc_z[n][tid]) * c - mx) * inv_sR;
     atomicAdd(&mass[v / SPAN], fmax(0.0, pv - static_cast<double>(q_s[tid])) - pv);
   }
   __syncthreads();
@@ -298,7 +300,7 @@ __global__ void __launch_bounds__(T2) reject_kernel(
     const int v = v0 + e;
     double rv = 0.0;
     if (v < V) {
-      rv = exp2(static_cast<double>(zr[v]) * c - mx) / sR;
+      rv = exp2(static_cast<double>(zr[v]) * c - mx) * inv_sR;
 #pragma unroll
       for (int k = 0; k < KC; ++k)
         if (cand_s[k] == v) rv = fmax(0.0, rv - static_cast<double>(q_s[k]));

@@ -497,8 +497,21 @@ def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, de
     del graphs
 
     # stage breakdown (after the timed region, same clocks regime): cycle k of
-    # one graph brackets stage BREAKDOWN[k % 5]
-    sg, sm = _graph_steps(step, len(BREAKDOWN) * BREAKDOWN_SAMPLES, lambda k: BREAKDOWN[k % len(BREAKDOWN)])
+    # one graph brackets stage BREAKDOWN[k % 5].  This graph is captured
+    # without programmatic launch: with it, a kernel may start before the
+    # event node in front of it, and a bracket of a few microseconds then
+    # misses part of its stage.  Each stage here runs serialised -- its own
+    # launch plus its execution -- an upper bound on what it adds to a
+    # pipelined cycle.
+    pdl_before = os.environ.get("DFLASH_PDL")
+    os.environ["DFLASH_PDL"] = "0"
+    try:
+        sg, sm = _graph_steps(step, len(BREAKDOWN) * BREAKDOWN_SAMPLES, lambda k: BREAKDOWN[k % len(BREAKDOWN)])
+    finally:
+        if pdl_before is None:
+            del os.environ["DFLASH_PDL"]
+        else:
+            os.environ["DFLASH_PDL"] = pdl_before
     sg.replay()
     torch.cuda.synchronize()
     if int(step.status.item()) != 0:
@@ -575,25 +588,20 @@ def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, de
                       "on a side branch of the graph so the kernels keep their programmatic launch; evenly spaced "
                       "cycles of every timed graph: at least %d samples (every cycle when the run has no more "
                       "steps), over the timed region" % LM_SAMPLES)
-    # the selection's cost in the cycle: (LM head + selection) - LM head, two
-    # long brackets (a bracket around the short selection alone is not
-    # reliable: its kernel may launch before the start event is recorded)
-    stages = {"conv2tap": 1e3 * stage_ms["conv2tap"], "lmhead_topk": 1e3 * stage_ms["lmhead_topk"],
-              "select_verify": 1e3 * sel_added_ms,
-              "select_verify_share": sel_added_ms / cyc_ms,
-              "select_verify_bracketed_alone": 1e3 * stage_ms["select_verify"],
+    stages = {**{n: 1e3 * stage_ms[n] for n in stage_ms},
+              "select_verify_share": stage_ms["select_verify"] / cyc_ms,
+              "select_verify_added": 1e3 * sel_added_ms,
+              "select_verify_added_share": sel_added_ms / cyc_ms,
               "event_pair_overhead": 1e3 * ev_ms,
               "samples": {n: len(samples[n]) for n in BREAKDOWN},
               "raw_us": {n: {k: (1e3 * v if k != "n" else v) for k, v in _summ(samples[n]).items()}
                          for n in BREAKDOWN},
-              "note": ("medians over one extra graph after the timed region whose cycle k brackets stage "
-                       "k mod 5 (%d samples per stage) with event nodes in the kernel chain, net of the two "
-                       "event nodes (measured alone); select_verify = (LM head + selection bracketed "
-                       "together) - (LM head bracketed alone): what selection and verification add to a "
-                       "cycle; select_verify_bracketed_alone is the selection bracketed by itself, for "
-                       "reference only (a few-microsecond bracket is not reliable: the bracketed kernel can "
-                       "be launched before the start event is recorded, so its samples split between its "
-                       "full time and a fraction of it)" % BREAKDOWN_SAMPLES)}
+              "note": ("medians over one extra graph after the timed region, captured without programmatic "
+                       "launch, whose cycle k brackets stage k mod 5 (%d samples per stage) with event nodes "
+                       "in the kernel chain, net of the two event nodes (measured alone): each stage's time is "
+                       "its own launch plus its execution, serialised -- an upper bound on what it adds to the "
+                       "pipelined cycles of the timed region; select_verify_added = (LM head + selection "
+                       "bracketed together) - (LM head bracketed alone)" % BREAKDOWN_SAMPLES)}
     config = {"workload": w.name + {"greedy": "", "sample": "+sampled-walk(T=1)",
                                     "ctx": "+context-gated-scorer"}[args.cycle]
                           + ("+dynamic-conv" if args.conv == "dynamic" else ""),

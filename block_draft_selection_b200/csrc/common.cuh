@@ -42,12 +42,11 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// On unless DFLASH_PDL=0 (read at every launch, so a caller can capture one
+// graph with and another without programmatic launch).
 inline bool pdl_enabled() {
-  static const bool on = [] {
-    const char* e = std::getenv("DFLASH_PDL");
-    return !(e != nullptr && e[0] == '0');
-  }();
-  return on;
+  const char* e = std::getenv("DFLASH_PDL");
+  return !(e != nullptr && e[0] == '0');
 }
 
 // Launch with programmatic stream serialisation (and an optional cluster

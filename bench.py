@@ -452,22 +452,29 @@ def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, de
     # roofline's launch duration has at least LM_SAMPLES samples from the
     # timed region (every cycle when there are no more steps than that) while
     # most cycles keep their kernel-to-kernel launch overlap
+    # The bracketed cycles alternate between the LM head alone and the LM
+    # head with the selection after it ("lmhead_select"): the difference of
+    # their medians is what the selection adds to a pipelined cycle.
+    span_name = lambda j: "lmhead_topk" if j % 2 == 0 else "lmhead_select"
     if args.eager:
         chunk, graphs = 1, []
-        marks = [{"lmhead_topk": (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))}
-                 for _ in range(steps)]
+        marks = [{span_name(k): (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))}
+                 for k in range(steps)]
     else:
         chunk = _chunk(steps)
         n_rep = steps // chunk
         n_graphs = min(64, n_rep)
-        per_graph = min(chunk, -(-LM_SAMPLES // n_graphs))
+        per_graph = min(chunk, -(-2 * LM_SAMPLES // n_graphs))
         spacing = chunk // per_graph
         # evenly spaced and centred: with one bracket per graph it sits in the
         # middle cycle (the last cycle of a graph measured about 10 us slower
         # at qwen3-4b-bs1 than the same stage anywhere else)
-        timed = {spacing // 2 + j * spacing for j in range(per_graph)}
-        graphs = [_graph_steps(step, chunk, lambda k: "lmhead_topk" if k in timed else None, side=True)
-                  for _ in range(n_graphs)]
+        timed = [spacing // 2 + j * spacing for j in range(per_graph)]
+
+        def plan(gi):
+            names = {k: span_name(gi * per_graph + j) for j, k in enumerate(timed)}
+            return lambda k: names.get(k)
+        graphs = [_graph_steps(step, chunk, plan(gi), side=True) for gi in range(n_graphs)]
         for g, _ in graphs:
             g.replay()              # one untimed replay of each captured graph
     barrier()
@@ -489,9 +496,11 @@ def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, de
     # LM-head launch durations of the timed region: every cycle of the eager
     # loop, or every cycle of each graph's last replay
     if args.eager:
-        lm_samples = [m["lmhead_topk"][0].elapsed_time(m["lmhead_topk"][1]) for m in marks]
+        spans = [(n, a.elapsed_time(b)) for m in marks for n, (a, b) in m.items()]
     else:
-        lm_samples = [a.elapsed_time(b) for _, gm in graphs for _, (a, b) in gm]
+        spans = [(n, a.elapsed_time(b)) for _, gm in graphs for n, (a, b) in gm]
+    lm_samples = [t for n, t in spans if n == "lmhead_topk"]
+    ls_samples = [t for n, t in spans if n == "lmhead_select"]
     ms_max = reduce_max(ms, world)
     value = aggregate(w.B, world, ms_max, steps)
     del graphs
@@ -528,6 +537,10 @@ def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, de
     # together) - (LM head bracketed alone); both gross, the event cost cancels
     sel_added_ms = max(0.0, med("lmhead_select") - med("lmhead_topk"))
     cyc_ms = ms_max / steps
+    # the same difference inside the timed region, where every kernel keeps
+    # its programmatic launch (side-branch brackets)
+    sel_pipe_ms = (max(0.0, statistics.median(ls_samples) - statistics.median(lm_samples))
+                   if ls_samples and lm_samples else None)
 
     # end-to-end leg: the library's DraftCycle, one graph launch per step that
     # copies the step's inputs from pinned host memory, runs the cycle and
@@ -586,12 +599,16 @@ def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, de
     roof["timing"] = ("mean CUDA-event duration of the LM-head call (GEMM+epilogue kernel and merge kernel), from "
                       "the completion of the kernel before it to the completion of its merge kernel; events recorded "
                       "on a side branch of the graph so the kernels keep their programmatic launch; evenly spaced "
-                      "cycles of every timed graph: at least %d samples (every cycle when the run has no more "
-                      "steps), over the timed region" % LM_SAMPLES)
+                      "cycles of every timed graph, alternating with brackets of the LM head + selection: at least "
+                      "%d samples of each (every other cycle when the run has too few steps for that), over the "
+                      "timed region" % LM_SAMPLES)
     stages = {**{n: 1e3 * stage_ms[n] for n in stage_ms},
               "select_verify_share": stage_ms["select_verify"] / cyc_ms,
               "select_verify_added": 1e3 * sel_added_ms,
               "select_verify_added_share": sel_added_ms / cyc_ms,
+              "select_verify_pipelined": None if sel_pipe_ms is None else 1e3 * sel_pipe_ms,
+              "select_verify_pipelined_share": None if sel_pipe_ms is None else sel_pipe_ms / cyc_ms,
+              "pipelined_samples": {"lmhead_topk": len(lm_samples), "lmhead_select": len(ls_samples)},
               "event_pair_overhead": 1e3 * ev_ms,
               "samples": {n: len(samples[n]) for n in BREAKDOWN},
               "raw_us": {n: {k: (1e3 * v if k != "n" else v) for k, v in _summ(samples[n]).items()}
@@ -601,7 +618,10 @@ def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, de
                        "in the kernel chain, net of the two event nodes (measured alone): each stage's time is "
                        "its own launch plus its execution, serialised -- an upper bound on what it adds to the "
                        "pipelined cycles of the timed region; select_verify_added = (LM head + selection "
-                       "bracketed together) - (LM head bracketed alone)" % BREAKDOWN_SAMPLES)}
+                       "bracketed together) - (LM head bracketed alone). select_verify_pipelined: the same "
+                       "difference of medians inside the timed region, where the brackets hang off the kernel "
+                       "chain on side branches and every kernel keeps its programmatic launch: what the "
+                       "selection adds to the timed cycles" % BREAKDOWN_SAMPLES)}
     config = {"workload": w.name + {"greedy": "", "sample": "+sampled-walk(T=1)",
                                     "ctx": "+context-gated-scorer"}[args.cycle]
                           + ("+dynamic-conv" if args.conv == "dynamic" else ""),

@@ -243,14 +243,14 @@ class Step:
             self.cws = torch.empty(max(1, bds.dflash_conv2tap_dynamic_workspace(w.B, w.P, w.d)),
                                    dtype=torch.uint8, device=dev)
         if cycle == "ctx":
-            # the pages' context-gated scorer: tied embeddings (the head), e = 256
+            # the pages' context-gated scorer: tied embeddings (the head), e = 256;
+            # the token tables A, B for the whole vocabulary are weights: built once
             Pab, Pg = syn.ctx_scorer_weights(w, 256)
             self.Pab, self.Pg = bds.bf16_tensor(Pab, dev), bds.bf16_tensor(Pg, dev)
             self.anchor = torch.from_numpy(syn.anchors(w.B, w.V, wr.seed)).to(dev)
-            self.proj = e((w.B * (1 + 16 * w.L), 512), torch.float32)
+            self.tab = bds.dflash_ctx_table(self.W, self.Pab)
             self.gate = e((w.M, 256), torch.float32)
-            self.pws = torch.empty(max(16, bds.dflash_ctx_project_workspace(w.B, w.L, w.d)), dtype=torch.uint8,
-                                   device=dev)
+            self.gate_stream = torch.cuda.Stream(device=dev)
         if cycle == "sample":
             # the target's logits at the L drafted positions and the bonus
             # position (the library's plain GEMM on the noised hidden states)
@@ -259,15 +259,16 @@ class Step:
             u = lambda shape, name: torch.from_numpy(syn.uniforms(shape, wr.seed, name)).to(dev)
             self.u_walk, self.u_acc, self.u_res = u((w.B, w.L), "u_walk"), u((w.B, w.L), "u_accept"), u((w.B,), "u_resample")
             self.q = e((w.B, w.L, 16), torch.float32)
-            self.rws = torch.empty(max(1, bds.dflash_verify_rejection_workspace(w.B, w.L, w.V)), dtype=torch.uint8,
+            self.rws = torch.empty(max(16, bds.dflash_verify_rejection_workspace(w.B, w.L, w.V)), dtype=torch.uint8,
                                    device=dev)
 
     # conv, LM-head GEMM+epilogue, LM-head merge, select+verify
     LAUNCHES_PER_STEP = 4
     # sample cycle: conv, LM head (2), walk, rejection verification (2)
     LAUNCHES_PER_STEP_SAMPLE = 6
-    # ctx cycle: conv, LM head (2), projections (gather + 2 GEMMs), scores + walk
-    LAUNCHES_PER_STEP_CTX = 7
+    # ctx cycle: conv, LM head (2), gate GEMM (its zeroing, when K is split, is
+    # a memset node, not a kernel), scores + walk
+    LAUNCHES_PER_STEP_CTX = 5
 
     def launches(self):
         n = {"sample": self.LAUNCHES_PER_STEP_SAMPLE, "ctx": self.LAUNCHES_PER_STEP_CTX}.get(
@@ -316,6 +317,13 @@ class Step:
                 put(ev[1])
 
         stage("event_pair", lambda: None)    # calibration: two event nodes, nothing between
+        if self.cycle == "ctx":
+            # the gate needs only H: it runs on a forked stream beside the conv
+            # and the LM head, and the walk waits for it
+            cur = self.torch.cuda.current_stream()
+            self.gate_stream.wait_stream(cur)
+            with self.torch.cuda.stream(self.gate_stream):
+                bds.dflash_ctx_gate(self.H, self.Pg, gate=self.gate)
         if self.conv == "dynamic":
             stage("conv2tap", lambda: bds.dflash_conv2tap_dynamic(self.x, self.a0, self.a1, self.Wc, self.prev,
                                                                   y=self.y, ws=self.cws))
@@ -338,9 +346,8 @@ class Step:
             stage("select_verify", walk_verify)
         elif self.cycle == "ctx":
             def ctx_select_verify():
-                bds.dflash_ctx_project(self.W, self.H, self.Pab, self.Pg, self.ix, self.anchor, self.w.B, self.w.L,
-                                       proj=self.proj, gate=self.gate, ws=self.pws, dev_status=self.status)
-                bds.dflash_ctx_walk(self.lp, self.ix, self.anchor, self.proj, self.gate, self.w.B, self.w.L,
+                self.torch.cuda.current_stream().wait_stream(self.gate_stream)
+                bds.dflash_ctx_walk(self.lp, self.ix, self.anchor, self.tab, self.gate, self.w.B, self.w.L,
                                     self.w.V, walk="maxsum", target=self.target, path_tok=self.tok,
                                     path_slot=self.slot, path_score=self.score, accept_len=self.acc,
                                     next_token=self.nxt, dev_status=self.status)
@@ -356,13 +363,17 @@ class Step:
 
 def _graph_steps(step, n_steps, plan, side=False):
     """Capture n_steps cycles into one CUDA graph.  plan(k) names the stage
-    whose call cycle k brackets with a pair of external timing events (event
-    nodes; in the kernel chain, or on a side branch with side=True), or
-    None.  Returns (graph, [(stage name, (start, end))])."""
+    (or a tuple of stages) whose call cycle k brackets with a pair of
+    external timing events (event nodes; in the kernel chain, or on a side
+    branch with side=True), or None.  Returns (graph, [(stage name, (start,
+    end))])."""
     import torch
     ev = lambda: (torch.cuda.Event(enable_timing=True, external=True),
                   torch.cuda.Event(enable_timing=True, external=True))
-    marks = [{plan(k): ev()} if plan(k) else None for k in range(n_steps)]
+    def names(k):
+        n = plan(k)
+        return () if not n else ((n,) if isinstance(n, str) else tuple(n))
+    marks = [{n: ev() for n in names(k)} or None for k in range(n_steps)]
     g = torch.cuda.CUDAGraph()
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
@@ -452,29 +463,22 @@ def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, de
     # roofline's launch duration has at least LM_SAMPLES samples from the
     # timed region (every cycle when there are no more steps than that) while
     # most cycles keep their kernel-to-kernel launch overlap
-    # The bracketed cycles alternate between the LM head alone and the LM
-    # head with the selection after it ("lmhead_select"): the difference of
-    # their medians is what the selection adds to a pipelined cycle.
-    span_name = lambda j: "lmhead_topk" if j % 2 == 0 else "lmhead_select"
     if args.eager:
         chunk, graphs = 1, []
-        marks = [{span_name(k): (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))}
-                 for k in range(steps)]
+        marks = [{"lmhead_topk": (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))}
+                 for _ in range(steps)]
     else:
         chunk = _chunk(steps)
         n_rep = steps // chunk
         n_graphs = min(64, n_rep)
-        per_graph = min(chunk, -(-2 * LM_SAMPLES // n_graphs))
+        per_graph = min(chunk, -(-LM_SAMPLES // n_graphs))
         spacing = chunk // per_graph
         # evenly spaced and centred: with one bracket per graph it sits in the
         # middle cycle (the last cycle of a graph measured about 10 us slower
         # at qwen3-4b-bs1 than the same stage anywhere else)
-        timed = [spacing // 2 + j * spacing for j in range(per_graph)]
-
-        def plan(gi):
-            names = {k: span_name(gi * per_graph + j) for j, k in enumerate(timed)}
-            return lambda k: names.get(k)
-        graphs = [_graph_steps(step, chunk, plan(gi), side=True) for gi in range(n_graphs)]
+        timed = {spacing // 2 + j * spacing for j in range(per_graph)}
+        graphs = [_graph_steps(step, chunk, lambda k: "lmhead_topk" if k in timed else None, side=True)
+                  for _ in range(n_graphs)]
         for g, _ in graphs:
             g.replay()              # one untimed replay of each captured graph
     barrier()
@@ -496,14 +500,28 @@ def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, de
     # LM-head launch durations of the timed region: every cycle of the eager
     # loop, or every cycle of each graph's last replay
     if args.eager:
-        spans = [(n, a.elapsed_time(b)) for m in marks for n, (a, b) in m.items()]
+        lm_samples = [m["lmhead_topk"][0].elapsed_time(m["lmhead_topk"][1]) for m in marks]
     else:
-        spans = [(n, a.elapsed_time(b)) for _, gm in graphs for n, (a, b) in gm]
-    lm_samples = [t for n, t in spans if n == "lmhead_topk"]
-    ls_samples = [t for n, t in spans if n == "lmhead_select"]
+        lm_samples = [a.elapsed_time(b) for _, gm in graphs for _, (a, b) in gm]
     ms_max = reduce_max(ms, world)
     value = aggregate(w.B, world, ms_max, steps)
     del graphs
+
+    # what the selection adds to a pipelined cycle (after the timed region):
+    # one graph whose cycles alternate side-branch brackets of the LM head
+    # alone and of the LM head with the selection after it, every kernel
+    # keeping its programmatic launch; the difference of the medians.  (Two
+    # brackets in one cycle would fork the chain between the LM head and the
+    # selection, which delays the selection.)
+    pg, pm = _graph_steps(step, 2 * LM_SAMPLES, lambda k: ("lmhead_topk", "lmhead_select")[k % 2], side=True)
+    pg.replay()
+    torch.cuda.synchronize()
+    if int(step.status.item()) != 0:
+        raise RuntimeError(f"device status {int(step.status.item())} in the pipelined brackets ({w.name})")
+    lmp = [a.elapsed_time(b) for n, (a, b) in pm if n == "lmhead_topk"]
+    lsp = [a.elapsed_time(b) for n, (a, b) in pm if n == "lmhead_select"]
+    del pg, pm
+    sel_pipe_ms = max(0.0, statistics.median(lsp) - statistics.median(lmp))
 
     # stage breakdown (after the timed region, same clocks regime): cycle k of
     # one graph brackets stage BREAKDOWN[k % 5].  This graph is captured
@@ -537,10 +555,7 @@ def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, de
     # together) - (LM head bracketed alone); both gross, the event cost cancels
     sel_added_ms = max(0.0, med("lmhead_select") - med("lmhead_topk"))
     cyc_ms = ms_max / steps
-    # the same difference inside the timed region, where every kernel keeps
-    # its programmatic launch (side-branch brackets)
-    sel_pipe_ms = (max(0.0, statistics.median(ls_samples) - statistics.median(lm_samples))
-                   if ls_samples and lm_samples else None)
+
 
     # end-to-end leg: the library's DraftCycle, one graph launch per step that
     # copies the step's inputs from pinned host memory, runs the cycle and
@@ -599,16 +614,15 @@ def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, de
     roof["timing"] = ("mean CUDA-event duration of the LM-head call (GEMM+epilogue kernel and merge kernel), from "
                       "the completion of the kernel before it to the completion of its merge kernel; events recorded "
                       "on a side branch of the graph so the kernels keep their programmatic launch; evenly spaced "
-                      "cycles of every timed graph, alternating with brackets of the LM head + selection: at least "
-                      "%d samples of each (every other cycle when the run has too few steps for that), over the "
-                      "timed region" % LM_SAMPLES)
+                      "cycles of every timed graph: at least %d samples (every cycle when the run has no more "
+                      "steps), over the timed region" % LM_SAMPLES)
     stages = {**{n: 1e3 * stage_ms[n] for n in stage_ms},
               "select_verify_share": stage_ms["select_verify"] / cyc_ms,
               "select_verify_added": 1e3 * sel_added_ms,
               "select_verify_added_share": sel_added_ms / cyc_ms,
-              "select_verify_pipelined": None if sel_pipe_ms is None else 1e3 * sel_pipe_ms,
-              "select_verify_pipelined_share": None if sel_pipe_ms is None else sel_pipe_ms / cyc_ms,
-              "pipelined_samples": {"lmhead_topk": len(lm_samples), "lmhead_select": len(ls_samples)},
+              "select_verify_pipelined": 1e3 * sel_pipe_ms,
+              "select_verify_pipelined_share": sel_pipe_ms / cyc_ms,
+              "pipelined_samples": {"lmhead_topk": len(lmp), "lmhead_select": len(lsp)},
               "event_pair_overhead": 1e3 * ev_ms,
               "samples": {n: len(samples[n]) for n in BREAKDOWN},
               "raw_us": {n: {k: (1e3 * v if k != "n" else v) for k, v in _summ(samples[n]).items()}
@@ -619,9 +633,9 @@ def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, de
                        "its own launch plus its execution, serialised -- an upper bound on what it adds to the "
                        "pipelined cycles of the timed region; select_verify_added = (LM head + selection "
                        "bracketed together) - (LM head bracketed alone). select_verify_pipelined: the same "
-                       "difference of medians inside the timed region, where the brackets hang off the kernel "
-                       "chain on side branches and every kernel keeps its programmatic launch: what the "
-                       "selection adds to the timed cycles" % BREAKDOWN_SAMPLES)}
+                       "difference of medians from a second extra graph whose cycles alternate the two brackets "
+                       "on side branches of the kernel chain, every kernel keeping its programmatic launch as in "
+                       "the timed region: what the selection adds to the timed cycles" % BREAKDOWN_SAMPLES)}
     config = {"workload": w.name + {"greedy": "", "sample": "+sampled-walk(T=1)",
                                     "ctx": "+context-gated-scorer"}[args.cycle]
                           + ("+dynamic-conv" if args.conv == "dynamic" else ""),

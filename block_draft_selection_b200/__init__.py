@@ -17,8 +17,8 @@ from ._binding import (  # noqa: F401
     dflash_conv2tap,
     dflash_conv2tap_dynamic,
     dflash_conv2tap_dynamic_workspace,
-    dflash_ctx_project,
-    dflash_ctx_project_workspace,
+    dflash_ctx_gate,
+    dflash_ctx_table,
     dflash_ctx_walk,
     dflash_gemm_bf16,
     dflash_lmhead_logits_debug,

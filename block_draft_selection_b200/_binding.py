@@ -56,11 +56,11 @@ def _load():
         "dflash_path_walk": (i32, [vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, i32, i32, i32, i32,
                                    vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "dflash_verify_rejection_workspace": (sz, [i32, i32, i32]),
-        "dflash_ctx_project_workspace": (sz, [i32, i32, i32]),
         "dflash_lmhead_topk_records": (i32, [i32, i32, i32]),
         "dflash_lmhead_topk_partial": (i32, [vp, vp, i32, i32, i32, i32, vp, sz, vp, vp]),
         "dflash_lmhead_topk_merge": (i32, [vp, i32, i32, i32, i32, vp, vp, vp, vp]),
-        "dflash_ctx_project": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, sz, vp, vp]),
+        "dflash_ctx_table": (i32, [vp, vp, i32, i32, i32, vp, vp]),
+        "dflash_ctx_gate": (i32, [vp, vp, i32, i32, i32, vp, vp]),
         "dflash_ctx_walk": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, ctypes.c_float,
                                   vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "dflash_verify_rejection": (i32, [vp, ctypes.c_float, vp, vp, vp, vp, vp, vp, i32, i32, i32,
@@ -369,7 +369,7 @@ def dflash_verify_rejection(target_logits, temperature, draft, draft_slot, cand_
     accept_len = _out(accept_len, "accept_len", torch.int32, (B,), dev)
     next_token = _out(next_token, "next_token", torch.int32, (B,), dev)
     if ws is None:
-        ws = torch.empty(max(1, dflash_verify_rejection_workspace(B, L, V)), dtype=torch.uint8, device=dev)
+        ws = torch.empty(max(16, dflash_verify_rejection_workspace(B, L, V)), dtype=torch.uint8, device=dev)
     _check("dflash_verify_rejection", lib.dflash_verify_rejection(
         _ptr(target_logits), float(temperature), _ptr(draft), _ptr(draft_slot), _ptr(cand_idx),
         _ptr(draft_q), _ptr(u_accept), _ptr(u_resample), B, L, V, _ptr(accept_len), _ptr(next_token),
@@ -377,38 +377,35 @@ def dflash_verify_rejection(target_logits, temperature, draft, draft_slot, cand_
     return accept_len, next_token
 
 
-def dflash_ctx_project_workspace(B: int, L: int, d: int) -> int:
-    return int(lib.dflash_ctx_project_workspace(B, L, d))
-
-
-def dflash_ctx_project(Emb, H, Pab, Pg, topk_idx, anchor, B, L, proj=None, gate=None, ws=None, dev_status=None,
-                       stream=None):
-    """Projections of the context-gated scorer: returns (proj [B*(1+16L), 2e] f32,
-    gate [B*L, e] f32, before the sigmoid)."""
+def dflash_ctx_table(Emb, Pab, tab=None, stream=None):
+    """A and B of the context-gated scorer for every token: tab [V, 2e] fp32
+    = Emb . Pab^T (row v: A(v), then B(v)).  Computed once per weight set."""
     _need(Emb, "Emb", torch.bfloat16)
     V, d = Emb.shape
-    _need(H, "H", torch.bfloat16, (B * L, d))
     _need(Pab, "Pab", torch.bfloat16)
     e = Pab.shape[0] // 2
     _need(Pab, "Pab", torch.bfloat16, (2 * e, d))
+    tab = _out(tab, "tab", torch.float32, (V, 2 * e), Emb.device)
+    _check("dflash_ctx_table", lib.dflash_ctx_table(_ptr(Emb), _ptr(Pab), V, d, e, _ptr(tab), _stream(stream)))
+    return tab
+
+
+def dflash_ctx_gate(H, Pg, gate=None, stream=None):
+    """The context gate before its sigmoid: gate [M, e] fp32 = H . Pg^T."""
+    _need(H, "H", torch.bfloat16)
+    M, d = H.shape
+    _need(Pg, "Pg", torch.bfloat16)
+    e = Pg.shape[0]
     _need(Pg, "Pg", torch.bfloat16, (e, d))
-    _need(topk_idx, "topk_idx", torch.int32, (B * L, K_TOP))
-    _need(anchor, "anchor", torch.int32, (B,))
-    dev = Emb.device
-    proj = _out(proj, "proj", torch.float32, (B * (1 + K_TOP * L), 2 * e), dev)
-    gate = _out(gate, "gate", torch.float32, (B * L, e), dev)
-    if ws is None:
-        ws = torch.empty(max(16, dflash_ctx_project_workspace(B, L, d)), dtype=torch.uint8, device=dev)
-    _check("dflash_ctx_project", lib.dflash_ctx_project(
-        _ptr(Emb), _ptr(H), _ptr(Pab), _ptr(Pg), _ptr(topk_idx), _ptr(anchor), B, L, V, d, e, _ptr(proj),
-        _ptr(gate), _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream)))
-    return proj, gate
+    gate = _out(gate, "gate", torch.float32, (M, e), H.device)
+    _check("dflash_ctx_gate", lib.dflash_ctx_gate(_ptr(H), _ptr(Pg), M, d, e, _ptr(gate), _stream(stream)))
+    return gate
 
 
 _WALKS = {"maxsum": 0, "greedy": 1, "sample": 2}
 
 
-def dflash_ctx_walk(topk_logp, topk_idx, anchor, proj, gate, B, L, V, walk="maxsum", uniforms=None,
+def dflash_ctx_walk(topk_logp, topk_idx, anchor, tab, gate, B, L, V, walk="maxsum", uniforms=None,
                     temperature=1.0, want_tables=False, target=None, path_tok=None, path_slot=None,
                     path_score=None, path_q=None, accept_len=None, next_token=None, dev_status=None, stream=None):
     """Scores of the context-gated scorer and a walk from the anchor.  Returns
@@ -420,8 +417,8 @@ def dflash_ctx_walk(topk_logp, topk_idx, anchor, proj, gate, B, L, V, walk="maxs
     _need(gate, "gate", torch.float32)
     e = gate.shape[1]
     _need(gate, "gate", torch.float32, (B * L, e))
-    _need(proj, "proj", torch.float32, (B * (1 + K_TOP * L), 2 * e))
-    dev = proj.device
+    _need(tab, "tab", torch.float32, (V, 2 * e))
+    dev = tab.device
     if walk == "sample":
         _need(uniforms, "uniforms", torch.float32, (B, L))
     path_tok = _out(path_tok, "path_tok", torch.int32, (B, L), dev)
@@ -436,7 +433,7 @@ def dflash_ctx_walk(topk_logp, topk_idx, anchor, proj, gate, B, L, V, walk="maxs
     else:
         accept_len = next_token = None
     _check("dflash_ctx_walk", lib.dflash_ctx_walk(
-        _ptr(topk_logp), _ptr(topk_idx), _ptr(anchor), _ptr(proj), _ptr(gate), B, L, K_TOP, e, V, _WALKS[walk],
+        _ptr(topk_logp), _ptr(topk_idx), _ptr(anchor), _ptr(tab), _ptr(gate), B, L, K_TOP, e, V, _WALKS[walk],
         _ptr(uniforms) if walk == "sample" else None, float(temperature), _ptr(path_tok), _ptr(path_slot),
         _ptr(path_score), _ptr(path_q), _ptr(tables), _ptr(target), _ptr(accept_len), _ptr(next_token),
         _ptr(dev_status), _stream(stream)))

@@ -7,12 +7,11 @@
 // Here A(a) = Pa.emb(a), B(b) = Pb.emb(b) (Pab = [Pa; Pb], [2e, d]),
 // H(h_t) = sigmoid(Pg.h_t) (Pg [e, d]) and U_t(b) the drafter's log-probability.
 //
-// dflash_ctx_project: the projections as GEMMs on the tensor cores.  A
-// gather kernel copies, per block, the anchor's embedding row and the 16 L
-// candidates' rows into a contiguous [B (1 + 16 L), d] buffer; then
-//   proj = rows . Pab^T   [B (1 + 16 L), 2e]   (A in columns 0..e-1, B in e..2e-1)
-//   gate = H . Pg^T       [B L, e]             (before the sigmoid)
-// with the library's tcgen05 GEMM.
+// A and B are functions of the token alone: dflash_ctx_table tabulates them
+// once for the whole vocabulary, tab = Emb . Pab^T [V, 2e], and a cycle only
+// reads the rows of its anchor and candidates.  dflash_ctx_gate computes
+// gate = H . Pg^T [B L, e] (before the sigmoid).  Both are the library's
+// tcgen05 GEMM.
 //
 // dflash_ctx_walk: one thread-block cluster of Q CTAs per block; CTA q scores
 // tables t = q, q+Q, ... (table t: predecessor = the anchor for t = 0, else
@@ -37,29 +36,6 @@ constexpr int THREADS = 256;
 constexpr int KC = 16;
 constexpr int MAX_CLUSTER = 8;
 constexpr int MAX_E = 1024;
-
-// rows per block in the projection buffers: the anchor, then 16 per position
-__host__ __device__ inline int rows_per_block(int L) { return 1 + KC * L; }
-
-__global__ void __launch_bounds__(256) gather_kernel(const uint4* __restrict__ Emb, const int32_t* __restrict__ topk_idx,
-                                                     const int32_t* __restrict__ anchor, int B, int L, int V, int d8,
-                                                     uint4* __restrict__ out, int* status) {
-  pdl_wait();
-  pdl_trigger();
-  const int R = rows_per_block(L);
-  const long long row = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (row >= static_cast<long long>(B) * R) return;
-  const int b = static_cast<int>(row / R);
-  const int o = static_cast<int>(row - static_cast<long long>(b) * R);
-  int tok = o == 0 ? __ldg(anchor + b) : __ldg(topk_idx + static_cast<size_t>(b) * L * KC + (o - 1));
-  if (tok < 0 || tok >= V) {
-    if ((threadIdx.x & 31) == 0) set_status(status, DFLASH_ERR_BAD_INDEX);
-    tok = 0;
-  }
-  const uint4* src = Emb + static_cast<size_t>(tok) * d8;
-  uint4* dst = out + static_cast<size_t>(row) * d8;
-  for (int c = threadIdx.x & 31; c < d8; c += 32) dst[c] = __ldg(src + c);
-}
 
 struct Layout {
   int ep;  // padded row length of the w / B buffers (floats)
@@ -91,7 +67,7 @@ __host__ __device__ inline Layout layout(int L, int e) {
 
 template <int WALK>
 __global__ void __launch_bounds__(THREADS) ctx_walk_kernel(
-    const float* __restrict__ topk_logp, const int32_t* __restrict__ topk_idx, const float* __restrict__ proj,
+    const float* __restrict__ topk_logp, const int32_t* __restrict__ topk_idx, const float* __restrict__ tab,
     const float* __restrict__ gate, int L, int e, int V, int Q, WalkArgs wa, int32_t* __restrict__ path_tok,
     int32_t* __restrict__ path_slot, float* __restrict__ path_score, float* __restrict__ tables_dbg,
     const int32_t* __restrict__ target, int32_t* __restrict__ accept_len, int32_t* __restrict__ next_token,
@@ -112,8 +88,8 @@ __global__ void __launch_bounds__(THREADS) ctx_walk_kernel(
   const int q_rank = blockIdx.x - b * Q;
   const int tid = threadIdx.x;
   const size_t row0 = static_cast<size_t>(b) * L;
-  const size_t prow0 = static_cast<size_t>(b) * rows_per_block(L);
   const int e4 = e / 4;
+  const size_t tw = 2 * static_cast<size_t>(e);   // floats per table row
   int pre_t = 0;
   float pre_u = 0.f;
   if (q_rank == 0 && tid < 32) {
@@ -125,9 +101,10 @@ __global__ void __launch_bounds__(THREADS) ctx_walk_kernel(
     S_out = cooperative_groups::this_cluster().map_shared_rank(Ss, 0);
     asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   }
-  if (q_rank == 0) {
+  {
     // the walk's tokens: internal position 0 = the anchor (16 copies), then
-    // the candidates of drafted positions 0..L-1
+    // the candidates of drafted positions 0..L-1 (every CTA: they pick the
+    // table rows; the leader's copy also feeds the walk)
     for (int q = tid; q < (L + 1) * KC; q += THREADS) {
       int c;
       if (q < KC) {
@@ -154,13 +131,14 @@ __global__ void __launch_bounds__(THREADS) ctx_walk_kernel(
     for (int q = tid; q < KC * e4; q += THREADS) {
       const int j = q / e4;
       const int c4 = q - j * e4;
-      const size_t prow = t == 0 ? prow0 : prow0 + 1 + static_cast<size_t>(t - 1) * KC + j;
-      const float4 a = __ldg(reinterpret_cast<const float4*>(proj + prow * (2 * e)) + c4);
+      // predecessor j: internal position t; successor j: internal position t + 1
+      const size_t prow = static_cast<size_t>(toks[t * KC + j]);
+      const size_t srow = static_cast<size_t>(toks[(t + 1) * KC + j]);
+      const float4 a = __ldg(reinterpret_cast<const float4*>(tab + prow * tw) + c4);
       const float4 g = *reinterpret_cast<const float4*>(gb + 4 * c4);
       *reinterpret_cast<float4*>(Wb + j * lo.ep + 4 * c4) = make_float4(a.x * g.x, a.y * g.y, a.z * g.z, a.w * g.w);
-      const size_t srow = prow0 + 1 + static_cast<size_t>(t) * KC + j;
       *reinterpret_cast<float4*>(Bb + j * lo.ep + 4 * c4) =
-          __ldg(reinterpret_cast<const float4*>(proj + srow * (2 * e) + e) + c4);
+          __ldg(reinterpret_cast<const float4*>(tab + srow * tw + e) + c4);
     }
     __syncthreads();
     {
@@ -207,7 +185,7 @@ __global__ void __launch_bounds__(THREADS) ctx_walk_kernel(
 }
 
 template <int WALK>
-static int launch_walk(const float* topk_logp, const int32_t* topk_idx, const float* proj, const float* gate, int B,
+static int launch_walk(const float* topk_logp, const int32_t* topk_idx, const float* tab, const float* gate, int B,
                        int L, int e, int V, WalkArgs wa, int32_t* path_tok, int32_t* path_slot, float* path_score,
                        float* tables_dbg, const int32_t* target, int32_t* accept_len, int32_t* next_token,
                        int* dev_status, cudaStream_t st) {
@@ -227,7 +205,7 @@ static int launch_walk(const float* topk_logp, const int32_t* topk_idx, const fl
     while (Q > 1 && static_cast<long long>(B) * Q > sms) --Q;
   }
   const cudaError_t e2 = launch_kernel_cluster(ctx_walk_kernel<WALK>, dim3(B * Q), dim3(THREADS), lo.total, st, Q,
-                                               topk_logp, topk_idx, proj, gate, L, e, V, Q, wa, path_tok, path_slot,
+                                               topk_logp, topk_idx, tab, gate, L, e, V, Q, wa, path_tok, path_slot,
                                                path_score, tables_dbg, target, accept_len, next_token, dev_status);
   return e2 == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }
@@ -235,59 +213,46 @@ static int launch_walk(const float* topk_logp, const int32_t* topk_idx, const fl
 }  // namespace ctx
 }  // namespace dflash
 
-extern "C" size_t dflash_ctx_project_workspace(int B, int L, int d) {
-  if (B < 1 || L < 1 || d < 1) return 0;
-  return static_cast<size_t>(B) * dflash::ctx::rows_per_block(L) * d * 2;
+extern "C" int dflash_ctx_table(const dflash_bf16* Emb, const dflash_bf16* Pab, int V, int d, int e, float* tab,
+                                void* stream) {
+  using namespace dflash::ctx;
+  if (!Emb || !Pab || !tab) return DFLASH_ERR_INVALID_ARG;
+  if (V < 1 || d < 8 || d % 8 != 0 || e < 16 || e > MAX_E || e % 8 != 0) return DFLASH_ERR_INVALID_ARG;
+  return dflash_gemm_bf16(Emb, Pab, tab, V, 2 * e, d, stream);
 }
 
-extern "C" int dflash_ctx_project(const dflash_bf16* Emb, const dflash_bf16* H, const dflash_bf16* Pab,
-                                  const dflash_bf16* Pg, const int32_t* topk_idx, const int32_t* anchor, int B, int L,
-                                  int V, int d, int e, float* proj, float* gate, void* ws, size_t ws_bytes,
-                                  int* dev_status, void* stream) {
+extern "C" int dflash_ctx_gate(const dflash_bf16* H, const dflash_bf16* Pg, int M, int d, int e, float* gate,
+                               void* stream) {
   using namespace dflash::ctx;
-  if (!Emb || !H || !Pab || !Pg || !topk_idx || !anchor || !proj || !gate) return DFLASH_ERR_INVALID_ARG;
-  if (B < 1 || L < 1 || L > 16 || V < 1 || d < 8 || d % 8 != 0 || e < 16 || e > MAX_E || e % 8 != 0)
-    return DFLASH_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(Emb) | reinterpret_cast<uintptr_t>(ws)) & 15) return DFLASH_ERR_INVALID_ARG;
-  const size_t need = dflash_ctx_project_workspace(B, L, d);
-  if (!ws || ws_bytes < need) return DFLASH_ERR_WORKSPACE;
-  const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const long long rows = static_cast<long long>(B) * rows_per_block(L);
-  if (rows > 0x7fffffffLL) return DFLASH_ERR_INVALID_ARG;
-  const int rows_per_cta = 8;
-  const cudaError_t ce = dflash::launch_kernel(
-      gather_kernel, dim3(static_cast<unsigned>((rows + rows_per_cta - 1) / rows_per_cta)), dim3(32 * rows_per_cta), 0,
-      st, reinterpret_cast<const uint4*>(Emb), topk_idx, anchor, B, L, V, d / 8, static_cast<uint4*>(ws), dev_status);
-  if (ce != cudaSuccess) return DFLASH_ERR_CUDA;
-  int rc = dflash_gemm_bf16(static_cast<const dflash_bf16*>(ws), Pab, proj, static_cast<int>(rows), 2 * e, d, stream);
-  if (rc != DFLASH_OK) return rc;
-  return dflash_gemm_bf16(H, Pg, gate, B * L, e, d, stream);
+  if (!H || !Pg || !gate) return DFLASH_ERR_INVALID_ARG;
+  if (M < 1 || d < 8 || d % 8 != 0 || e < 16 || e > MAX_E || e % 8 != 0) return DFLASH_ERR_INVALID_ARG;
+  return dflash_gemm_bf16(H, Pg, gate, M, e, d, stream);
 }
 
 extern "C" int dflash_ctx_walk(const float* topk_logp, const int32_t* topk_idx, const int32_t* anchor,
-                               const float* proj, const float* gate, int B, int L, int K, int e, int V, int walk,
+                               const float* tab, const float* gate, int B, int L, int K, int e, int V, int walk,
                                const float* uniforms, float temperature, int32_t* path_tok, int32_t* path_slot,
                                float* path_score, float* path_q, float* tables_dbg, const int32_t* target,
                                int32_t* accept_len, int32_t* next_token, int* dev_status, void* stream) {
   using namespace dflash::ctx;
-  if (!topk_logp || !topk_idx || !anchor || !proj || !gate || !path_tok) return DFLASH_ERR_INVALID_ARG;
+  if (!topk_logp || !topk_idx || !anchor || !tab || !gate || !path_tok) return DFLASH_ERR_INVALID_ARG;
   if (K != KC || B < 1 || L < 1 || L > 16 || V < 1 || e < 16 || e > MAX_E || e % 8 != 0)
     return DFLASH_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(proj) | reinterpret_cast<uintptr_t>(gate)) & 15) return DFLASH_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(tab) | reinterpret_cast<uintptr_t>(gate)) & 15) return DFLASH_ERR_INVALID_ARG;
   if (target && (!accept_len || !next_token)) return DFLASH_ERR_INVALID_ARG;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   WalkArgs wa{anchor, uniforms, 0.f, path_q};
   switch (walk) {
     case 0:
-      return launch_walk<WALK_VITERBI>(topk_logp, topk_idx, proj, gate, B, L, e, V, wa, path_tok, path_slot,
+      return launch_walk<WALK_VITERBI>(topk_logp, topk_idx, tab, gate, B, L, e, V, wa, path_tok, path_slot,
                                        path_score, tables_dbg, target, accept_len, next_token, dev_status, st);
     case 1:
-      return launch_walk<WALK_GREEDY>(topk_logp, topk_idx, proj, gate, B, L, e, V, wa, path_tok, path_slot,
+      return launch_walk<WALK_GREEDY>(topk_logp, topk_idx, tab, gate, B, L, e, V, wa, path_tok, path_slot,
                                       path_score, tables_dbg, target, accept_len, next_token, dev_status, st);
     case 2:
       if (!uniforms || !(temperature > 0.f) || !(temperature < INFINITY)) return DFLASH_ERR_INVALID_ARG;
       wa.inv_t = 1.f / temperature;
-      return launch_walk<WALK_SAMPLE>(topk_logp, topk_idx, proj, gate, B, L, e, V, wa, path_tok, path_slot,
+      return launch_walk<WALK_SAMPLE>(topk_logp, topk_idx, tab, gate, B, L, e, V, wa, path_tok, path_slot,
                                       path_score, tables_dbg, target, accept_len, next_token, dev_status, st);
     default:
       return DFLASH_ERR_INVALID_ARG;

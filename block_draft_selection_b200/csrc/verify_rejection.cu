@@ -13,16 +13,19 @@
 //
 // Two kernels:
 //   1. row statistics: CTA (row, slice) reduces 8192 logits of one row to
-//      (m, s) with c = log2(e) / T: m = c * max z, s = sum of
-//      exp2((z - max z) * c) (fp32 exponentials added in pairs in fp32, the
-//      pair sums in fp64) -- also the slice's probability mass once the row
-//      is merged;
-//   2. one CTA of 1024 threads per block: merges its L+1 rows' statistics,
-//      tests the L drafts (one lane each), picks the residual's slice from
-//      the slice masses (corrected at the 16 candidates), then scans that
-//      slice's 8192 entries with a block-wide fp64 prefix sum.  Every value
-//      that decides an outcome here (p at a draft token, the entries of the
-//      scanned slice) is an fp64 exponential.
+//      (m, s) with c = log2(e) / T: m = c * max z (the slice's max, found
+//      first), s = sum of exp2((z - max z) * c) (fp32 exponentials added in
+//      pairs in fp32, the pair sums in fp64) -- also the slice's probability
+//      mass once the row is merged;
+//   2. one CTA of 1024 threads per block: merges its L+1 rows' statistics
+//      (a warp per row: the max over the slices, then one fp64 rescale per
+//      slice), tests the L drafts (one lane each), picks the residual's slice
+//      from the slice masses (corrected at the 16 candidates), then scans
+//      that slice's 8192 entries with a block-wide fp64 prefix sum: each
+//      thread loads its 8 logits before any arithmetic and tests its range
+//      against the 16 candidates once.  Every value that decides an outcome
+//      here (p at a draft token, the entries of the scanned slice) is an
+//      fp64 exponential.
 #include <climits>
 
 #include "common.cuh"
@@ -44,21 +47,6 @@ struct Part {  // statistics of one slice of one row (16 bytes)
   double m;    // max of z*c over the slice (-inf: empty)
   double s;    // sum of exp2(z*c - m)
 };
-
-__device__ __forceinline__ void merge_ms(double& m, double& s, double m2, double s2) {
-  if (m2 == -INFINITY) return;
-  if (m == -INFINITY) {
-    m = m2;
-    s = s2;
-    return;
-  }
-  if (m2 > m) {
-    s = s * exp2(m - m2) + s2;
-    m = m2;
-  } else {
-    s += s2 * exp2(m2 - m);
-  }
-}
 
 __global__ void __launch_bounds__(T1) row_stats_kernel(const float* __restrict__ z, int V, int S, double c, int vec,
                                                        Part* __restrict__ part) {
@@ -88,10 +76,20 @@ __global__ void __launch_bounds__(T1) row_stats_kernel(const float* __restrict__
       x[j] = v < V ? __ldg(zr + v) : -INFINITY;
     }
   }
+  // the slice's maximum first (fp32, exact), then every exponential against it
+  __shared__ float wmax[T1 / 32];
+  __shared__ double wsum[T1 / 32];
+  const int warp = tid >> 5, lane = tid & 31;
   float xm = -INFINITY;
 #pragma unroll
   for (int j = 0; j < EPT1; ++j) xm = fmaxf(xm, x[j]);
-  double m = static_cast<double>(xm) * c;  // c > 0: the max of z*c is at the max of z
+#pragma unroll
+  for (int off = 16; off; off >>= 1) xm = fmaxf(xm, __shfl_xor_sync(FULL, xm, off));
+  if (lane == 0) wmax[warp] = xm;
+  __syncthreads();
+  xm = wmax[0];
+#pragma unroll
+  for (int w = 1; w < T1 / 32; ++w) xm = fmaxf(xm, wmax[w]);
   double s = 0.0;
   if (xm != -INFINITY) {
     // exp2((x - xm) * c) in fp32; neighbouring pairs added in fp32 (one
@@ -106,32 +104,22 @@ __global__ void __launch_bounds__(T1) row_stats_kernel(const float* __restrict__
       s += static_cast<double>(exp2f((x[j] - xm) * cf) + exp2f((x[j + 1] - xm) * cf));   // padding: 0
   }
 #pragma unroll
-  for (int off = 16; off; off >>= 1) {
-    const double m2 = __shfl_xor_sync(FULL, m, off);
-    const double s2 = __shfl_xor_sync(FULL, s, off);
-    merge_ms(m, s, m2, s2);
-  }
-  __shared__ double wm[T1 / 32];
-  __shared__ double wsum[T1 / 32];
-  const int warp = tid >> 5, lane = tid & 31;
-  if (lane == 0) {
-    wm[warp] = m;
-    wsum[warp] = s;
-  }
+  for (int off = 16; off; off >>= 1) s += __shfl_xor_sync(FULL, s, off);
+  if (lane == 0) wsum[warp] = s;
   __syncthreads();
   if (tid == 0) {
-    double mb = wm[0];
-    double sb = wsum[0];
-    for (int w = 1; w < T1 / 32; ++w) merge_ms(mb, sb, wm[w], wsum[w]);
+    double sb = 0.0;
+#pragma unroll
+    for (int w = 0; w < T1 / 32; ++w) sb += wsum[w];
     Part p;
-    p.m = mb;
+    p.m = static_cast<double>(xm) * c;   // c > 0: the max of z*c is at the max of z
     p.s = sb;
     part[row * S + split] = p;
   }
 }
 
 __global__ void __launch_bounds__(T2) reject_kernel(
-    const float* __restrict__ z, int V, int S, double c, int L, const Part* __restrict__ part,
+    const float* __restrict__ z, int V, int S, double c, int vec, int L, const Part* __restrict__ part,
     const int32_t* __restrict__ draft, const int32_t* __restrict__ draft_slot, const int32_t* __restrict__ cand_idx,
     const float* __restrict__ draft_q, const float* __restrict__ u_accept, const float* __restrict__ u_resample,
     int32_t* __restrict__ accept_len, int32_t* __restrict__ next_token, int* status) {
@@ -193,21 +181,25 @@ __global__ void __launch_bounds__(T2) reject_kernel(
     pc_z[i][k] = zv;
   }
 
-  // A. each row's max and sum from its slices (warp i -> row i)
+  // A. each row's max and sum from its slices (warp i -> row i; lane j holds
+  // slices j and j + 32): the warp's max first, then one rescale per slice
   if (warp <= L) {
-    double m = -INFINITY;
+    Part p0{-INFINITY, 0.0}, p1{-INFINITY, 0.0};
+    const Part* pr = part + (row0 + warp) * S;
+    if (lane < S) p0 = pr[lane];
+    if (lane + 32 < S) p1 = pr[lane + 32];
+    if (lane < S) parts_s[warp][lane] = p0;
+    if (lane + 32 < S) parts_s[warp][lane + 32] = p1;
+    double m = fmax(p0.m, p1.m);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) m = fmax(m, __shfl_xor_sync(FULL, m, off));
     double s = 0.0;
-    for (int j = lane; j < S; j += 32) {
-      const Part p = part[(row0 + warp) * S + j];
-      parts_s[warp][j] = p;
-      merge_ms(m, s, p.m, p.s);
+    if (m != -INFINITY) {
+      if (p0.m != -INFINITY) s += p0.s * exp2(p0.m - m);
+      if (p1.m != -INFINITY) s += p1.s * exp2(p1.m - m);
     }
 #pragma unroll
-    for (int off = 16; off; off >>= 1) {
-      const double m2 = __shfl_xor_sync(FULL, m, off);
-      const double s2 = __shfl_xor_sync(FULL, s, off);
-      merge_ms(m, s, m2, s2);
-    }
+    for (int off = 16; off; off >>= 1) s += __shfl_xor_sync(FULL, s, off);
     if (lane == 0) {
       row_m[warp] = m;
       row_s[warp] = s;
@@ -288,10 +280,27 @@ __global__ void __launch_bounds__(T2) reject_kernel(
   }
   __syncthreads();
 
-  // E. inverse CDF inside the slice: block-wide prefix sum of the residual
+  // E. inverse CDF inside the slice: block-wide prefix sum of the residual.
+  // Each thread's 8 consecutive logits are loaded before any arithmetic (as
+  // two 16-byte loads where the row allows it), and its range is tested
+  // against the 16 candidates once.
   const int js = sh_slice;
   const double target = sh_target;
   const int v0 = js * SPAN + tid * EPT2;
+  float zv[EPT2];
+  if (vec) {
+    // V % 4 == 0 and v0 % 8 == 0: a quad that starts inside the row ends inside it
+    const float4 lo = v0 < V ? __ldg(reinterpret_cast<const float4*>(zr + v0)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 hi = v0 + 4 < V ? __ldg(reinterpret_cast<const float4*>(zr + v0 + 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    zv[0] = lo.x; zv[1] = lo.y; zv[2] = lo.z; zv[3] = lo.w;
+    zv[4] = hi.x; zv[5] = hi.y; zv[6] = hi.z; zv[7] = hi.w;
+  } else {
+#pragma unroll
+    for (int e = 0; e < EPT2; ++e) zv[e] = v0 + e < V ? __ldg(zr + v0 + e) : 0.f;
+  }
+  bool has_cand = false;
+#pragma unroll
+  for (int k = 0; k < KC; ++k) has_cand |= static_cast<unsigned>(cand_s[k] - v0) < static_cast<unsigned>(EPT2);
   double r[EPT2];
   double tsum = 0.0;
   int last_pos = -1;
@@ -300,10 +309,15 @@ __global__ void __launch_bounds__(T2) reject_kernel(
     const int v = v0 + e;
     double rv = 0.0;
     if (v < V) {
-      rv = exp2(static_cast<double>(zr[v]) * c - mx) * inv_sR;
+      rv = exp2(static_cast<double>(zv[e]) * c - mx) * inv_sR;
+      if (has_cand) {
+        // which candidate (if any) is entry v: integer selects only, then
+        // one fp64 correction (the candidates are distinct)
+        int hit = -1;
 #pragma unroll
-      for (int k = 0; k < KC; ++k)
-        if (cand_s[k] == v) rv = fmax(0.0, rv - static_cast<double>(q_s[k]));
+        for (int k = 0; k < KC; ++k) hit = cand_s[k] == v ? k : hit;
+        if (hit >= 0) rv = fmax(0.0, rv - static_cast<double>(q_s[hit]));
+      }
     }
     r[e] = rv;
     tsum += rv;
@@ -386,7 +400,7 @@ extern "C" int dflash_verify_rejection(const float* target_logits, float tempera
   cudaError_t e = dflash::launch_kernel(row_stats_kernel, dim3(rows, S), dim3(T1), 0, st, target_logits, V, S, c,
                                         vec, part);
   if (e != cudaSuccess) return DFLASH_ERR_CUDA;
-  e = dflash::launch_kernel(reject_kernel, dim3(B), dim3(T2), 0, st, target_logits, V, S, c, L,
+  e = dflash::launch_kernel(reject_kernel, dim3(B), dim3(T2), 0, st, target_logits, V, S, c, vec, L,
                             static_cast<const Part*>(part), draft, draft_slot, cand_idx, draft_q, u_accept,
                             u_resample, accept_len, next_token, dev_status);
   return e == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;

@@ -11,8 +11,9 @@
  *   dflash_path_walk        greedy or sampled walk from the last verified token
  *   dflash_verify_rejection rejection-sampling verification against the
  *                           target's distributions
- *   dflash_ctx_project,     the pages' context-gated pair scorer: its
- *   dflash_ctx_walk         projections, then its scores and a walk
+ *   dflash_ctx_table,       the pages' context-gated pair scorer: its
+ *   dflash_ctx_gate,        token tables, its gate, then its scores and a
+ *   dflash_ctx_walk         walk
  *
  * Sources: "DFlash 2: Keep Drafting Parallel" (the blog, read in its Chinese
  * translation) and "Inco AI's DFlash 2 lifts LLM decoding output 16-25%".
@@ -307,8 +308,9 @@ int dflash_path_walk(const float* topk_logp, const int32_t* topk_idx, const dfla
  * (distinct per row); draft_q [B, L, 16] fp32; u_accept [B, L] and
  * u_resample [B] fp32 uniforms in [0, 1).  accept_len, next_token [B] int32
  * out.  ws: device workspace of dflash_verify_rejection_workspace(B, L, V)
- * bytes, 16-byte aligned.  1 <= L <= 31, 1 <= V <= 524288.  A draft token or
- * slot out of range records DFLASH_ERR_BAD_INDEX and is clamped.
+ * bytes, 16-byte aligned (the slice statistics; no initial contents needed).
+ * 1 <= L <= 31, 1 <= V <= 524288.  A draft token or slot out of range
+ * records DFLASH_ERR_BAD_INDEX and is clamped.
  */
 size_t dflash_verify_rejection_workspace(int B, int L, int V);
 int dflash_verify_rejection(const float* target_logits, float temperature, const int32_t* draft,
@@ -318,28 +320,26 @@ int dflash_verify_rejection(const float* target_logits, float temperature, const
                             int* dev_status, void* stream);
 
 /*
- * The pages' context-gated pair scorer, part 1: projections.
+ * The pages' context-gated pair scorer, part 1: the token tables and the gate.
  * "DFlash 2: Keep Drafting Parallel", section "a lightweight path selector":
  * S_t(a, b) = U_t(b) + <A(a) (.) H(h_t), B(b)>, compact token embeddings A, B
  * matched under a context gate H.  Read here as A(a) = Pa.emb(a),
  * B(b) = Pb.emb(b), H(h_t) = sigmoid(Pg.h_t), emb(v) = Emb[v].
  *
- * Emb [V, d] bf16 (16-byte aligned), H [B*L, d] bf16 (the drafted positions'
- * hidden states), Pab [2e, d] bf16 (rows 0..e-1 = Pa, e..2e-1 = Pb), Pg [e, d]
- * bf16, topk_idx [B*L, 16] int32, anchor [B] int32 (last verified token).
- * Outputs: proj [B*(1+16L), 2e] fp32 -- per block, row 0 = the anchor, row
- * 1 + 16t + k = candidate k of position t; columns 0..e-1 = A, e..2e-1 = B --
- * and gate [B*L, e] fp32 = Pg.h (before the sigmoid).
- * ws: dflash_ctx_project_workspace(B, L, d) bytes (16-byte aligned; the
- * gathered embedding rows).  1 <= L <= 16, d % 8 == 0, 16 <= e <= 1024,
- * e % 8 == 0.  A token index outside [0, V) is read as 0 and records
- * DFLASH_ERR_BAD_INDEX.
+ * A and B depend on the token alone, so they are tabulated once for the whole
+ * vocabulary (whenever Emb or Pab change) and every cycle only reads rows:
+ *   dflash_ctx_table: tab [V, 2e] fp32 = Emb . Pab^T -- row v holds A(v) in
+ *     columns 0..e-1 and B(v) in columns e..2e-1.  Emb [V, d] bf16, Pab
+ *     [2e, d] bf16 (rows 0..e-1 = Pa, e..2e-1 = Pb).
+ *   dflash_ctx_gate: gate [M, e] fp32 = H . Pg^T (before the sigmoid), H
+ *     [M = B*L, d] bf16 (the drafted positions' hidden states), Pg [e, d]
+ *     bf16.  It needs only H, so a caller can run it on another stream
+ *     while the LM head runs.
+ * Both run on the library's tensor-core GEMM (dflash_gemm_bf16; its rules
+ * on alignment apply).  d % 8 == 0, 16 <= e <= 1024, e % 8 == 0.
  */
-size_t dflash_ctx_project_workspace(int B, int L, int d);
-int dflash_ctx_project(const dflash_bf16* Emb, const dflash_bf16* H, const dflash_bf16* Pab,
-                       const dflash_bf16* Pg, const int32_t* topk_idx, const int32_t* anchor, int B, int L,
-                       int V, int d, int e, float* proj, float* gate, void* ws, size_t ws_bytes,
-                       int* dev_status, void* stream);
+int dflash_ctx_table(const dflash_bf16* Emb, const dflash_bf16* Pab, int V, int d, int e, float* tab, void* stream);
+int dflash_ctx_gate(const dflash_bf16* H, const dflash_bf16* Pg, int M, int d, int e, float* gate, void* stream);
 
 /*
  * The pages' context-gated pair scorer, part 2: scores and a walk from the
@@ -350,13 +350,14 @@ int dflash_ctx_project(const dflash_bf16* Emb, const dflash_bf16* H, const dflas
  * constant that no walk's choice depends on).  walk: 0 = max-sum from the
  * anchor (ties: lowest slot), 1 = greedy, 2 = sampled at `temperature` with
  * one uniform per drafted position (as dflash_path_walk).
- * Inputs from dflash_lmhead_topk and dflash_ctx_project; proj, gate 16-byte
- * aligned.  Outputs: path_tok [B, L]; path_slot [B, L], path_score [B]
+ * Inputs from dflash_lmhead_topk, dflash_ctx_table (tab [V, 2e]) and
+ * dflash_ctx_gate; tab, gate 16-byte aligned.  A token index outside [0, V)
+ * is read as 0 and records DFLASH_ERR_BAD_INDEX.  Outputs: path_tok [B, L]; path_slot [B, L], path_score [B]
  * (the sum of the chosen entries), path_q [B, L, 16] (sampling only) and
  * tables_dbg [B, L, 16, 16] are nullable; target [B, L+1] (nullable) adds
  * greedy verification into accept_len, next_token [B].  K must be 16.
  */
-int dflash_ctx_walk(const float* topk_logp, const int32_t* topk_idx, const int32_t* anchor, const float* proj,
+int dflash_ctx_walk(const float* topk_logp, const int32_t* topk_idx, const int32_t* anchor, const float* tab,
                     const float* gate, int B, int L, int K, int e, int V, int walk, const float* uniforms,
                     float temperature, int32_t* path_tok, int32_t* path_slot, float* path_score, float* path_q,
                     float* tables_dbg, const int32_t* target, int32_t* accept_len, int32_t* next_token,

@@ -109,17 +109,17 @@ def test_host_side_rejections(lib):
     assert lib.dflash_lmhead_topk_merge(fake, 4, 148, 2, 15, fake, fake, None, None) == 1
     assert lib.dflash_lmhead_topk_merge(fake, 4, 0, 2, 16, fake, fake, None, None) == 1
     assert lib.dflash_lmhead_topk_merge(fake, 4, 148, 0, 16, fake, fake, None, None) == 1
-    # context-gated scorer: e not a multiple of 8, L > 16, K != 16, unknown walk, sampling without uniforms
+    # context-gated scorer: e not a multiple of 8 or out of range, d not a multiple of 8, K != 16, unknown
+    # walk, sampling without uniforms
     i32 = ctypes.c_int
-    lib.dflash_ctx_project.argtypes = [vp] * 6 + [i32] * 5 + [vp, vp, vp, ctypes.c_size_t, vp, vp]
-    assert lib.dflash_ctx_project(fake, fake, fake, fake, fake, fake, 1, 4, 100, 256, 20, fake, fake, fake, big,
-                                  None, None) == 1
-    assert lib.dflash_ctx_project(fake, fake, fake, fake, fake, fake, 1, 17, 100, 256, 32, fake, fake, fake, big,
-                                  None, None) == 1
-    assert lib.dflash_ctx_project(fake, fake, fake, fake, fake, fake, 1, 4, 100, 256, 32, fake, fake, fake,
-                                  ctypes.c_size_t(16), None, None) == 4
-    lib.dflash_ctx_project_workspace.restype = ctypes.c_size_t
-    assert lib.dflash_ctx_project_workspace(2, 3, 64) == 2 * 49 * 64 * 2
+    lib.dflash_ctx_table.argtypes = [vp, vp, i32, i32, i32, vp, vp]
+    assert lib.dflash_ctx_table(fake, fake, 100, 256, 20, fake, None) == 1
+    assert lib.dflash_ctx_table(fake, fake, 100, 250, 32, fake, None) == 1
+    assert lib.dflash_ctx_table(fake, fake, 100, 256, 1032, fake, None) == 1
+    assert lib.dflash_ctx_table(None, fake, 100, 256, 32, fake, None) == 1
+    lib.dflash_ctx_gate.argtypes = [vp, vp, i32, i32, i32, vp, vp]
+    assert lib.dflash_ctx_gate(fake, fake, 4, 256, 12, fake, None) == 1
+    assert lib.dflash_ctx_gate(fake, fake, 0, 256, 32, fake, None) == 1
     lib.dflash_ctx_walk.argtypes = [vp] * 5 + [i32] * 6 + [vp, f32] + [vp] * 10
     walk = lambda K, walkid, u, T: lib.dflash_ctx_walk(fake, fake, fake, fake, fake, 1, 4, K, 32, 100, walkid, u, T,
                                                        fake, None, None, None, None, None, None, None, None, None)

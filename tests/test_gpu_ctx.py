@@ -1,7 +1,8 @@
 """The pages' context-gated pair scorer on the GPU against the oracle.
 
 Scores: every table entry within an a priori bound of the oracle's fp64
-value (the projections are fp32-accumulated GEMMs of exact bf16 products;
+value (the token tables A, B for the whole vocabulary and the gate are
+fp32-accumulated GEMMs of exact bf16 products;
 the gate's sigmoid and the e-term dot product add fp32 roundings).  Walks:
 the path must equal the oracle's where the oracle's margin allows it --
 max-sum: best minus second-best path score >= 1e-3; greedy: every step's
@@ -32,9 +33,9 @@ def _run(Emb, H, Pab, Pg, logp, idx, anchor, B, L, V, walk="maxsum", u=None, T=1
     import block_draft_selection_b200 as bds
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
-    proj, gate = bds.dflash_ctx_project(dev_bf16(Emb), dev_bf16(H), dev_bf16(Pab), dev_bf16(Pg), t(idx), t(anchor),
-                                        B, L, dev_status=status)
-    out = bds.dflash_ctx_walk(t(logp), t(idx), t(anchor), proj, gate, B, L, V, walk=walk,
+    tab = bds.dflash_ctx_table(dev_bf16(Emb), dev_bf16(Pab))
+    gate = bds.dflash_ctx_gate(dev_bf16(H), dev_bf16(Pg))
+    out = bds.dflash_ctx_walk(t(logp), t(idx), t(anchor), tab, gate, B, L, V, walk=walk,
                               uniforms=None if u is None else t(u), temperature=T, want_tables=True,
                               target=None if target is None else t(target), dev_status=status)
     torch.cuda.synchronize()
@@ -177,3 +178,28 @@ def test_ctx_edge_shapes(B, L, V, d, e):
         firm = ref["margin"] >= 1e-3 if walk == "maxsum" else (ref["margin"] >= 1e-3).all(axis=1)
         assert firm.mean() > 0.5
         np.testing.assert_array_equal(slot[firm], ref["path_slot"][firm])
+
+
+@pytest.mark.parametrize("name,e", [("qwen3-4b-bs1", 256), ("tiny", 64)])
+def test_ctx_table_rows(name, e):
+    """dflash_ctx_table against the exact products on sampled rows (the first
+    and last row of every 128-row tile and random ones), under the GEMM's
+    a priori fp32 bound; the gate likewise on every row."""
+    import block_draft_selection_b200 as bds
+    from block_draft_synth import bf16_bits_to_f32
+    w = syn.workload(name)
+    Emb, H, Pab, Pg, _, _, _ = _inputs(w, e)
+    f = lambda b: bf16_bits_to_f32(b).astype(np.float64)
+    tab = bds.dflash_ctx_table(dev_bf16(Emb), dev_bf16(Pab)).cpu().numpy()
+    gate = bds.dflash_ctx_gate(dev_bf16(H), dev_bf16(Pg)).cpu().numpy()
+    assert tab.shape == (w.V, 2 * e) and gate.shape == (w.M, e)
+    rng = np.random.default_rng(5)
+    rows = sorted({r for t0 in range(0, w.V, 128) for r in (t0, min(w.V, t0 + 128) - 1)}
+                  | set(rng.integers(0, w.V, 64).tolist()))
+    x, P = f(Emb[rows]), f(Pab)
+    d = x.shape[1]
+    exact = x @ P.T
+    bound = 4 * d * 2.0 ** -23 * (np.abs(x) @ np.abs(P).T) + 1e-6
+    assert (np.abs(tab[rows] - exact) <= bound).all()
+    xh, G = f(H), f(Pg)
+    assert (np.abs(gate - xh @ G.T) <= 4 * d * 2.0 ** -23 * (np.abs(xh) @ np.abs(G).T) + 1e-6).all()

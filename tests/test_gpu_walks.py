@@ -230,3 +230,52 @@ def test_verify_rejection_bad_index_is_reported():
                                 t(d["ua"]), t(d["ur"]), dev_status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 6
+
+
+def test_verify_rejection_workspace_reuse_and_masked_slices():
+    """One workspace over several calls of different batch sizes gives the
+    results of a fresh workspace each time.  Rows whose logits are -inf
+    outside a few slices (whole slices without mass, a slice with mass in its
+    first 232 entries only) still give valid draws."""
+    import block_draft_selection_b200 as bds
+    L, V, T = 5, 40000, 1.0
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    Bmax = 12
+    n_ws = bds.dflash_verify_rejection_workspace(Bmax, L, V)
+    ws = torch.full((n_ws,), 0xAB, dtype=torch.uint8, device="cuda")    # no initial contents needed
+    for B, seed in ((Bmax, 21), (3, 22), (Bmax, 21), (7, 23)):
+        d = _verify_inputs(B, L, V, seed, T)
+        z = d["z"].reshape(B, L + 1, V)
+        if seed == 23:
+            # every row keeps mass only in [8192, 16384) and [32768, 33000) (the drafts' raised logits aside)
+            keep = np.zeros(V, bool)
+            keep[8192:16384] = True
+            keep[32768:33000] = True
+            cand = d["idx"].reshape(B, L, 16)
+            for b in range(B):
+                for i in range(L + 1):
+                    m = keep.copy()
+                    if i < L:
+                        m[cand[b, i]] = True
+                    z[b, i, ~m] = -np.inf
+        d["z"] = z.reshape(B * (L + 1), V)
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        args = (t(d["z"]), T, t(d["draft"]), t(d["slot"]), t(d["idx"]), t(d["q"]), t(d["ua"]), t(d["ur"]))
+        acc, nxt = bds.dflash_verify_rejection(*args, ws=ws, dev_status=status)
+        acc2, nxt2 = bds.dflash_verify_rejection(*args, dev_status=status)     # a fresh workspace
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        np.testing.assert_array_equal(acc.cpu().numpy(), acc2.cpu().numpy())
+        np.testing.assert_array_equal(nxt.cpu().numpy(), nxt2.cpu().numpy())
+        acc, nxt = acc.cpu().numpy(), nxt.cpu().numpy()
+        p = oracle.target_probs(d["z"], T).reshape(B, L + 1, V)
+        cand = d["idx"].reshape(B, L, 16)
+        for b in range(B):
+            n = acc[b] - 1
+            if n == L:
+                res = p[b, L]
+            else:
+                qv = np.zeros(V)
+                qv[cand[b, n]] = d["q"][b, n]
+                res = np.maximum(0.0, p[b, n] - qv)
+            assert _valid_draw(res, float(d["ur"][b]), int(nxt[b]), 1e-6), (B, seed, b, nxt[b])

@@ -136,8 +136,6 @@ __global__ void __launch_bounds__(T2) reject_kernel(
   __shared__ float pc_q[MAX_L][KC];    // read up front (the rejected position is not yet
   __shared__ float pc_z[MAX_L][KC];    // known, and these loads need not wait for it)
 
-  pdl_wait();
-  pdl_trigger();
   const int b = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t row0 = static_cast<size_t>(b) * (L + 1);
@@ -146,10 +144,15 @@ __global__ void __launch_bounds__(T2) reject_kernel(
     sh_before = -1;
     sh_last = -1;
   }
+  // The drafts, their candidates and probabilities, the uniforms and the
+  // target logits are read before the dependency wait, while the statistics
+  // kernel runs: each of its CTAs starts this kernel only after its own wait
+  // on the kernel before it, so all of these are complete and visible here.
   // warp 0, lane i < L: drafted position i's token, slot, q and target logit
   int dx = 0;
   double dq = 0.0, du = 0.0;
   float dz = 0.f;
+  const float ures = warp == 0 ? u_resample[b] : 0.f;   // used in D
   if (warp == 0 && lane < L) {
     const size_t di = static_cast<size_t>(b) * L + lane;
     dx = draft[di];
@@ -180,6 +183,8 @@ __global__ void __launch_bounds__(T2) reject_kernel(
     pc_q[i][k] = draft_q[ci];
     pc_z[i][k] = zv;
   }
+  pdl_wait();   // the slice statistics
+  pdl_trigger();
 
   // A. each row's max and sum from its slices (warp i -> row i; lane j holds
   // slices j and j + 32): the warp's max first, then one rescale per slice
@@ -258,7 +263,7 @@ __global__ void __launch_bounds__(T2) reject_kernel(
     }
     const double excl = incl - (m0 + m1);
     const double total = __shfl_sync(FULL, incl, 31);
-    const double target = static_cast<double>(u_resample[b]) * total;
+    const double target = static_cast<double>(ures) * total;
     const unsigned over = __ballot_sync(FULL, incl > target);
     const unsigned pos = __ballot_sync(FULL, m0 > 0.0 || m1 > 0.0);
     if (lane == 0) sh_target = target;

@@ -146,8 +146,10 @@ __global__ void __launch_bounds__(T2) reject_kernel(
   }
   // The drafts, their candidates and probabilities, the uniforms and the
   // target logits are read before the dependency wait, while the statistics
-  // kernel runs: each of its CTAs starts this kernel only after its own wait
-  // on the kernel before it, so all of these are complete and visible here.
+  // kernel runs: this kernel starts only once every statistics CTA has
+  // triggered it, which each does after its own wait on the kernel before
+  // it, so all of these are complete and visible here (without programmatic
+  // launch the statistics kernel has simply finished).
   // warp 0, lane i < L: drafted position i's token, slot, q and target logit
   int dx = 0;
   double dq = 0.0, du = 0.0;

@@ -203,3 +203,28 @@ def test_ctx_table_rows(name, e):
     assert (np.abs(tab[rows] - exact) <= bound).all()
     xh, G = f(H), f(Pg)
     assert (np.abs(gate - xh @ G.T) <= 4 * d * 2.0 ** -23 * (np.abs(xh) @ np.abs(G).T) + 1e-6).all()
+
+
+def test_ctx_bad_index_is_reported():
+    """A candidate or anchor index outside [0, V) records DFLASH_ERR_BAD_INDEX
+    (it is read as token 0, and the call still returns a path of candidates)."""
+    import block_draft_selection_b200 as bds
+    w = syn.workload("tiny")
+    e = 32
+    Emb, H, Pab, Pg, logp, idx, anchor = _inputs(w, e)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    tab = bds.dflash_ctx_table(dev_bf16(Emb), dev_bf16(Pab))
+    gate = bds.dflash_ctx_gate(dev_bf16(H), dev_bf16(Pg))
+    for bad_idx, bad_anchor in ((True, False), (False, True)):
+        ix = idx.copy()
+        an = anchor.copy()
+        if bad_idx:
+            ix.reshape(-1)[5] = w.V + 7
+        if bad_anchor:
+            an[0] = -3
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        tok, slot, *_ = bds.dflash_ctx_walk(t(logp), t(ix), t(an), tab, gate, w.B, w.L, w.V, dev_status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == bds.DFLASH_ERR_BAD_INDEX
+        s = slot.cpu().numpy()
+        assert ((s >= 0) & (s < 16)).all()

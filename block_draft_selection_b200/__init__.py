@@ -39,7 +39,7 @@ from ._binding import (  # noqa: F401
     lib,
     workspace,
 )
-from .cycle import DraftCycle  # noqa: F401,E402
+from .cycle import DraftCycle, DraftPipeline  # noqa: F401,E402
 from .parallel import VocabParallelLMHead, vocab_shard  # noqa: F401,E402
 
 

@@ -16,6 +16,10 @@ results, and `run()` raises if the status is nonzero.  The conv does not feed
 the LM head, so its lane (one copy of its inputs in, the conv, one copy of its
 output out) runs on a second stream inside the same graph, overlapping the
 LM head; the step ends when both lanes have.
+
+`launch()` / `wait()` split `run()` in two, and DraftPipeline steps two
+cycles over the same weights alternately on two streams, for independent
+batches whose copies and kernels may overlap.
 """
 from __future__ import annotations
 
@@ -110,6 +114,7 @@ class DraftCycle:
         self.status = dv["status"]
         self.ws = b.workspace(M, V, d, dev)
         self._side = torch.cuda.Stream(device=dev)
+        self._done = None
         self._graph = None
         if use_graph:
             self._capture()
@@ -160,11 +165,26 @@ class DraftCycle:
         results.  Raises DFlashError when a kernel of the step recorded a
         device-side error (a bounded wait that ran out, a token index out of
         range): the results of such a step are not valid."""
-        if self._graph is not None:
-            self._graph.replay()
-        else:
-            self._step()
-        torch.cuda.current_stream().synchronize()
+        self.launch()
+        return self.wait()
+
+    def launch(self, stream=None):
+        """Enqueue one step on `stream` (the current stream if None) without
+        waiting for it; self.host_in must not change until wait() returns."""
+        stream = stream or torch.cuda.current_stream()
+        with torch.cuda.stream(stream):
+            if self._graph is not None:
+                self._graph.replay()
+            else:
+                self._step()
+            if self._done is None:
+                self._done = torch.cuda.Event()
+            self._done.record(stream)
+
+    def wait(self):
+        """Wait for the step launch() enqueued and return its host results
+        (raises DFlashError as run() does)."""
+        self._done.synchronize()
         code = int(self.host_out["status"][0])
         if code != 0:
             raise b.DFlashError("DraftCycle.run", code)
@@ -174,3 +194,50 @@ class DraftCycle:
         """Bytes a step copies host-to-device and device-to-host (both lanes'
         arenas, alignment padding included)."""
         return (int(self._hin.numel() + self._chin.numel()), int(self._hout.numel() + self._chout.numel()))
+
+
+class DraftPipeline:
+    """Two DraftCycles over the same device-resident weights, stepping
+    independent batches alternately on two streams, so that one batch's
+    copies overlap the other's kernels.  Step i runs on cycle i % 2: its host
+    inputs are filled after that cycle's previous step has been waited for,
+    and every step's results are read back to the host.  For serving
+    independent groups of blocks; a loop whose next inputs depend on the
+    previous step's results uses DraftCycle.run()."""
+
+    def __init__(self, W, E, Msel, a0, a1, B: int, L: int, P: int):
+        self.cycles = [DraftCycle(W, E, Msel, a0, a1, B, L, P) for _ in range(2)]
+        self.streams = [torch.cuda.Stream(device=W.device) for _ in range(2)]
+        self._pending = [False, False]
+        self._i = 0
+
+    def host_in(self):
+        """The host input views of the next step's cycle; waits for that
+        cycle's previous step and returns its results first (None if none)."""
+        k = self._i % 2
+        prev = None
+        if self._pending[k]:
+            prev = self.cycles[k].wait()
+            self._pending[k] = False
+        return self.cycles[k].host_in, prev
+
+    def launch(self):
+        """Enqueue the next step (its inputs filled through host_in())."""
+        k = self._i % 2
+        if self._pending[k]:
+            raise RuntimeError("DraftPipeline.launch: call host_in() first")
+        self.cycles[k].launch(self.streams[k])
+        self._pending[k] = True
+        self._i += 1
+
+    def drain(self):
+        """Wait for the steps still in flight, oldest first; their results."""
+        out = []
+        for j in (self._i % 2, (self._i + 1) % 2):
+            if self._pending[j]:
+                out.append(self.cycles[j].wait())
+                self._pending[j] = False
+        return out
+
+    def io_bytes(self):
+        return self.cycles[0].io_bytes()

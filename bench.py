@@ -396,6 +396,10 @@ def _chunk(steps, cap=32):
 
 # LM-head launch durations sampled inside the timed region (at least).
 LM_SAMPLES = 20
+# Samples of each bracket in the graph that measures what the selection adds
+# to a pipelined cycle (the difference of two medians of event spans a few
+# microseconds apart needs more than the roofline's mean).
+PIPE_SAMPLES = 40
 
 # Stage breakdown: one extra graph after the timed region in which cycle k
 # brackets stage BREAKDOWN[k % 5]; every stage gets BREAKDOWN_SAMPLES samples.
@@ -513,7 +517,7 @@ def measure(args, w: syn.Workload, steps, warmup: int, rank: int, world: int, de
     # keeping its programmatic launch; the difference of the medians.  (Two
     # brackets in one cycle would fork the chain between the LM head and the
     # selection, which delays the selection.)
-    pg, pm = _graph_steps(step, 2 * LM_SAMPLES, lambda k: ("lmhead_topk", "lmhead_select")[k % 2], side=True)
+    pg, pm = _graph_steps(step, 2 * PIPE_SAMPLES, lambda k: ("lmhead_topk", "lmhead_select")[k % 2], side=True)
     pg.replay()
     torch.cuda.synchronize()
     if int(step.status.item()) != 0:

@@ -299,7 +299,8 @@ int dflash_path_walk(const float* topk_logp, const int32_t* topk_idx, const dfla
  *   and next_token[b] is drawn from max(0, p_n - q_n) (n < L) or from p_L
  *   (n = L) by inverse CDF in vocabulary order: the smallest token whose
  *   cumulative mass exceeds u_resample[b] times the total mass.
- * The draw happens in fp64 on fp32 exponentials; a uniform that falls within
+ * The draw's 8192-token slice is chosen from fp64 sums of fp32 exponentials
+ * and the token inside it from fp64 exponentials; a uniform that falls within
  * about 1e-7 (relative) of a cumulative boundary may land on either side.
  *
  * target_logits [B*(L+1), V] fp32 (finite or -inf); temperature > 0 (the
